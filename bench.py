@@ -1,0 +1,460 @@
+#!/usr/bin/env python
+"""GPTQ layer quantization throughput on B200: weights quantized per second.
+
+One step = the whole GPTQ path for one LLaMA-7B-shaped q_proj layer
+(W 4096x4096, 262144 calibration tokens, 4-bit asymmetric, one scale per
+output channel, B = 128): zero H, accumulate H = 2 X X^T over all tokens,
+damp + factor to G, quantize + pack all columns.  Inputs are resident in HBM
+when the timed region starts (X is 2.1 GB, larger than L2).  With N GPUs
+every rank quantizes its own independent layer (weak scaling, no collective
+on the data path).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+from datetime import timedelta
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "GPTQ weights quantized/s per linear layer"
+UNIT = "weights/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
+                  "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=5)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", choices=["q_proj", "small"], default="q_proj")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def workload_spec(name: str, rank: int):
+    from post_weight_quantization_26_b200 import synth
+    base = synth.Q_PROJ_7B if name == "q_proj" else synth.SMALL_256
+    # weak scaling: every rank gets its own independent layer
+    return base.with_(w_seed=base.w_seed + rank, x_seed=base.x_seed + 100 * rank)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines: list[str] = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.dev)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=5)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------- oracle baseline
+def oracle_sample(spec, x_host, w_host, tokens=8192, rows=32):
+    """Time the CPU oracle on a bounded sample of the workload and scale to
+    one full layer: Hessian on a token prefix (scaled by n / prefix), the full
+    fp64 factorization, GPTQ on a subset of rows (scaled by d_row / rows)."""
+    import numpy as np
+
+    from oracle import gptq_oracle as O
+    t0 = time.perf_counter()
+    xs = x_host[:tokens].float().numpy()
+    h = O.hessian(xs)
+    t_h = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    hd, dead = O.dampen(h, spec.damp)
+    u = O.hinv_cholesky_upper(hd)
+    t_f = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    O.gptq_quantize(w_host[:rows].numpy().astype(np.float64), u, spec.bits, spec.group,
+                    spec.sym, spec.block, dead=dead)
+    t_q = time.perf_counter() - t0
+    total = t_h * spec.n_tokens / tokens + t_f + t_q * spec.d_row / rows
+    return {"seconds_per_layer": total, "hessian_s": t_h, "factor_s": t_f, "quant_s": t_q,
+            "sample": (f"H on {tokens} of {spec.n_tokens} tokens (x{spec.n_tokens / tokens:g}), "
+                       f"full {spec.d_col}^2 fp64 factorization, GPTQ on {rows} of "
+                       f"{spec.d_row} rows (x{spec.d_row / rows:g})")}
+
+
+def cpu_cores():
+    cores = len(os.sched_getaffinity(0))
+    try:
+        from threadpoolctl import threadpool_info
+        th = max((i.get("num_threads", 1) for i in threadpool_info()), default=cores)
+        return min(cores, th) if th else cores
+    except Exception:
+        return cores
+
+
+# --------------------------------------------------------------- reference
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    from post_weight_quantization_26_b200 import synth
+    spec = workload_spec(args.workload, 0)
+    tokens = min(8192, spec.n_tokens)
+    x_host = synth.gen_tokens(spec, 0, tokens)
+    w_host = synth.gen_weight(spec)
+    times = []
+    res = None
+    for i in range(args.warmup + args.steps):
+        res = oracle_sample(spec, x_host, w_host, tokens=tokens)
+        if i >= args.warmup:
+            times.append(res["seconds_per_layer"])
+    sec = statistics.mean(times)
+    value = spec.d_row * spec.d_col / sec
+    cores = cpu_cores()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(spec, world=1),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": res["sample"]},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(spec, world):
+    return {"workload": spec.name, "d_row": spec.d_row, "d_col": spec.d_col,
+            "n_tokens": spec.n_tokens, "bits": spec.bits, "group_size": spec.group,
+            "sym": spec.sym, "block": spec.block, "damp": spec.damp,
+            "w": f"{spec.w_dist} sigma={spec.w_sigma} {'bf16' if spec.w_bf16 else 'fp32'}",
+            "x": f"{spec.x_dist} bf16, {spec.outlier_count} channels x{spec.outlier_scale:g}",
+            "l2": "inputs larger than L2 (X bf16 %.2f GB)" % (spec.n_tokens * spec.d_col * 2 / 1e9),
+            "parallelism": f"{world} independent layer(s), one per GPU"}
+
+
+# ------------------------------------------------------------------- ours
+def kernel_traffic(name: str, src_rel: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current source of the kernel (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)[name]
+        with open(os.path.join(ROOT, src_rel), "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+        if rec.get("source_sha256") != sha:
+            return None
+        return rec["bytes_per_launch"]
+    except (OSError, KeyError, ValueError):
+        return None
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from post_weight_quantization_26_b200 import build as _build
+    from post_weight_quantization_26_b200 import gptq as G
+    from post_weight_quantization_26_b200 import synth
+
+    if rank == 0:
+        _build.build()
+    if world > 1:
+        dist.barrier()
+    G.load_library()
+    dev = torch.device("cuda", local_rank)
+    spec = workload_spec(args.workload, rank)
+    d, n, dr = spec.d_col, spec.n_tokens, spec.d_row
+    cfg = G.make_config(bits=spec.bits, group_size=spec.group, sym=spec.sym,
+                        block=spec.block, damp_rel=spec.damp)
+
+    x_host = torch.empty((n, d), dtype=torch.bfloat16).pin_memory()
+    synth.gen_tokens(spec, out=x_host)
+    w_host = synth.gen_weight(spec).pin_memory()
+    x = x_host.to(dev)
+    w = w_host.to(dev)
+    H = torch.zeros((d, d), dtype=torch.float32, device=dev)
+    Gm = torch.empty_like(H)
+    dead = torch.empty(d, dtype=torch.uint8, device=dev)
+    ws = G.alloc_workspace(dr, d, cfg, device=dev)
+    qw, sc, ze = G.alloc_outputs(dr, d, cfg, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        H.zero_()
+        if ev:
+            ev[1].record(stream)
+        G.gptq_hessian_accumulate(H, x)
+        if ev:
+            ev[2].record(stream)
+        G.gptq_prepare_hinv(H, spec.damp, Gm, dead, ws)
+        if ev:
+            ev[3].record(stream)
+        G.gptq_quantize_layer(w, Gm, dead, cfg, qw, sc, ze, ws)
+        if ev:
+            ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if G.gptq_device_status() != 0:
+        raise RuntimeError("device status set during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    launches0 = G.gptq_launch_count()
+    t0.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    launches = G.gptq_launch_count() - launches0
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    ms = t0.elapsed_time(t1) / args.steps
+    stages = {"zero_h": [], "hessian": [], "prepare": [], "quantize": []}
+    for e in evs:
+        stages["zero_h"].append(e[0].elapsed_time(e[1]))
+        stages["hessian"].append(e[1].elapsed_time(e[2]))
+        stages["prepare"].append(e[2].elapsed_time(e[3]))
+        stages["quantize"].append(e[3].elapsed_time(e[4]))
+    stage_ms = {k: statistics.mean(v) for k, v in stages.items()}
+    if G.gptq_device_status() != 0:
+        raise RuntimeError("device status set during the timed region")
+
+    ms_max = ms
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+    value = world * dr * d / (ms_max / 1e3)
+
+    # ---- end to end: host buffers in, host buffers out, through the same API
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, G, spec, cfg, x_host, w_host, dev, stream, world)
+
+    if rank != 0:
+        return
+    peaks, peak_src = load_peaks()
+    syrk_s = stage_ms["hessian"] / 1e3
+    syrk_flops = d * (d + 1) * n
+    achieved = syrk_flops / syrk_s / 1e12
+    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    traffic = kernel_traffic("syrk_bf16_tcgen05_kernel",
+                             "post_weight_quantization_26_b200/csrc/syrk_tcgen05.cuh")
+    roofline = {"bound": "tensor", "kernel": "syrk_bf16_tcgen05_kernel",
+                "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": traffic,
+                "peak_source": f"bf16_tflops_sustained of {peak_src}"}
+    # other stages against their own bounds (SM clock from the sampled median)
+    sm_mhz = (clk or {}).get("sm_mhz") or peaks.get("sm_max_mhz", 1965.0)
+    fp64_peak = 148 * 64 * 2 * sm_mhz * 1e6 / 1e12
+    fp32_peak = 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+    chol_flops = 2.0 / 3.0 * d ** 3
+    prop_flops = dr * d * (d - 1)
+    t_star = (syrk_flops / (peak * 1e12) + chol_flops / (fp64_peak * 1e12)
+              + prop_flops / (fp32_peak * 1e12)
+              + dr * d * (1 + spec.bits / 8) / (peaks.get("hbm_gbs", 6650.0) * 1e9))
+    stage_roofline = {
+        "hessian": {"ms": stage_ms["hessian"], "frac": achieved / peak, "bound": "tensor bf16"},
+        "prepare": {"ms": stage_ms["prepare"],
+                    "frac": chol_flops / (stage_ms["prepare"] / 1e3) / 1e12 / fp64_peak,
+                    "bound": f"alu fp64 {fp64_peak:.1f} TF/s at {sm_mhz:.0f} MHz"},
+        "quantize": {"ms": stage_ms["quantize"],
+                     "frac": prop_flops / (stage_ms["quantize"] / 1e3) / 1e12 / fp32_peak,
+                     "bound": f"alu fp32 {fp32_peak:.1f} TF/s at {sm_mhz:.0f} MHz"},
+        "zero_h": {"ms": stage_ms["zero_h"]},
+        "combined_t_star_ms": t_star * 1e3,
+        "combined_frac": t_star * 1e3 / ms,
+    }
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        res = oracle_sample(spec, x_host, w_host)
+        cpu = {"value": dr * d / res["seconds_per_layer"], "unit": UNIT, "cores": cpu_cores(),
+               "kind": "oracle", "sample": res["sample"],
+               "stage_s": {"hessian_full_est": res["hessian_s"] * n / 8192,
+                           "factor": res["factor_s"], "quant_full_est": res["quant_s"] * dr / 32}}
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 in / f32 acc (H); f64 (factor); f32 (sweep)",
+        "data": "synthetic (seeded LLaMA-7B-shaped layer and activations)",
+        "config": workload_config(spec, world),
+        "stage_ms": stage_ms, "stages": stage_roofline,
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": launches, "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, G, spec, cfg, x_host, w_host, dev, stream, world):
+    """Same metric through the public API with host buffers: every step copies
+    X (in chunks, overlapped with the accumulation on a copy stream) and W
+    from pinned host memory and reads the packed result back to the host."""
+    import torch
+    import torch.distributed as dist
+    d, n, dr = spec.d_col, spec.n_tokens, spec.d_row
+    chunk = 32768
+    stage = [torch.empty((chunk, d), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    copy_stream = torch.cuda.Stream(dev)
+    H = torch.zeros((d, d), dtype=torch.float32, device=dev)
+    Gm = torch.empty_like(H)
+    dead = torch.empty(d, dtype=torch.uint8, device=dev)
+    ws = G.alloc_workspace(dr, d, cfg, device=dev)
+    qw, sc, ze = G.alloc_outputs(dr, d, cfg, device=dev)
+    w = torch.empty((dr, d), dtype=torch.float32, device=dev)
+    qh = torch.empty(qw.shape, dtype=qw.dtype).pin_memory()
+    sh = torch.empty(sc.shape, dtype=sc.dtype).pin_memory()
+    zh = torch.empty(ze.shape, dtype=ze.dtype).pin_memory()
+    copied = [torch.cuda.Event() for _ in range(2)]
+    consumed = [torch.cuda.Event() for _ in range(2)]
+
+    def step():
+        H.zero_()
+        w.copy_(w_host, non_blocking=True)
+        nchunks = (n + chunk - 1) // chunk
+        for i in range(nchunks):
+            b = i & 1
+            a, e = i * chunk, min(n, (i + 1) * chunk)
+            with torch.cuda.stream(copy_stream):
+                if i >= 2:
+                    copy_stream.wait_event(consumed[b])
+                stage[b][: e - a].copy_(x_host[a:e], non_blocking=True)
+                copied[b].record(copy_stream)
+            stream.wait_event(copied[b])
+            G.gptq_hessian_accumulate(H, stage[b][: e - a])
+            consumed[b].record(stream)
+        G.gptq_prepare_hinv(H, spec.damp, Gm, dead, ws)
+        G.gptq_quantize_layer(w, Gm, dead, cfg, qw, sc, ze, ws)
+        qh.copy_(qw, non_blocking=True)
+        sh.copy_(sc, non_blocking=True)
+        zh.copy_(ze, non_blocking=True)
+
+    steps = max(1, args.steps)
+    for _ in range(max(1, min(args.warmup, 2))):
+        step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = t0.elapsed_time(t1) / steps
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    h2d = n * d * 2 + dr * d * 4
+    d2h = qw.numel() * 4 + sc.numel() * 4 + ze.numel()
+    return {"value": world * dr * d / (ms / 1e3), "unit": UNIT, "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

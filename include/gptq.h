@@ -1,0 +1,176 @@
+/*
+ * gptq.h -- C ABI of the B200 (sm_100a) GPTQ layer quantizer, libgptq.so.
+ *
+ * The method is GPTQ as described on the dingiv.github.io quantization page,
+ * section GPTQ: for one linear layer W (d_row x d_col, out x in) and
+ * calibration inputs X (d_col x n), find quantized W^ minimising
+ * ||W X - W^ X||_F^2 using the Hessian H = 2 X X^T, the upper Cholesky factor
+ * of H^-1, a fixed left-to-right column order, and blocks of B columns with
+ * immediate in-block error updates and one lazy batched update of the columns
+ * to the right after each block.  Output is b-bit codes (b = 2, 3, 4) with a
+ * scale and zero point per output channel or per group of input columns
+ * (granularity as on the psvmc.cn page, section 按量化粒度划分).
+ *
+ * Conventions for every call:
+ *  - All array pointers are DEVICE pointers owned by the caller; the library
+ *    allocates no device memory.  Scratch space comes from a caller-provided
+ *    workspace of gptq_workspace_size() bytes, 256-byte aligned.
+ *  - Matrices are dense row-major with the leading dimension stated.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default).
+ *  - Calls validate their arguments first; on GPTQ_ERR_INVALID or
+ *    GPTQ_ERR_WORKSPACE nothing is launched and no output is written.
+ *  - gptq_hessian_accumulate and gptq_quantize_layer are asynchronous and do
+ *    not synchronize.  gptq_prepare_hinv and gptq_dequant_check synchronize
+ *    `stream` once to return a status / value.
+ *  - Kernels never spin without bound.  A kernel whose internal wait runs out
+ *    records GPTQ_ERR_TIMEOUT in a device status word, frees what it holds
+ *    and returns; gptq_device_status() (or the next synchronizing call)
+ *    reports it.
+ */
+#ifndef GPTQ_B200_H
+#define GPTQ_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GPTQ_OK = 0,
+  GPTQ_ERR_INVALID = 1,    /* bad argument: null pointer, size, alignment, config */
+  GPTQ_ERR_NOT_SPD = 2,    /* damped H is not positive definite (see bad_pivot) */
+  GPTQ_ERR_NONFINITE = 3,  /* NaN or Inf found in H (prepare) */
+  GPTQ_ERR_WORKSPACE = 4,  /* workspace null, misaligned or smaller than required */
+  GPTQ_ERR_CUDA = 5,       /* a CUDA runtime call or launch failed */
+  GPTQ_ERR_TIMEOUT = 6     /* a kernel's bounded internal wait ran out */
+} gptq_status;
+
+/* Quantizer settings.
+ *  bits        2, 3 or 4.
+ *  group_size  0 = one scale/zero per output channel, computed from the
+ *              original row of W; otherwise the number of consecutive input
+ *              columns sharing a scale/zero, computed from the current
+ *              (error-updated) weights when the group's first column is
+ *              reached.  Must be a multiple of 32 that divides d_col, with
+ *              block % group_size == 0 or group_size % block == 0.
+ *  sym         0: asymmetric, codes q = clip(rint(w/s) + z, 0, 2^b-1) with
+ *                 s = (max(0,max w) - min(0,min w)) / (2^b-1), z = rint(-min(0,min w)/s);
+ *              1: symmetric, s = max|w| / (2^(b-1)-1), z = 2^(b-1) (codes
+ *                 stored offset-binary, i.e. signed code + 2^(b-1)).
+ *              Dequantized value: s * (q - z).  (dingiv.github.io page,
+ *              section 量化基础; youleyou.com page, sections 二 and 四.)
+ *  block       B, columns per lazy-update block: 32, 64 or 128.
+ *  damp_rel    relative damping: lambda = damp_rel * mean(diag H).
+ */
+typedef struct {
+  int bits;
+  int group_size;
+  int sym;
+  int block;
+  double damp_rel;
+} gptq_config;
+
+/* Bytes of workspace needed by gptq_prepare_hinv (d = d_col),
+ * gptq_quantize_layer and gptq_dequant_check for this layer shape: the
+ * maximum over the three.  Returns 0 if the arguments are invalid. */
+size_t gptq_workspace_size(int64_t d_row, int64_t d_col, const gptq_config* cfg);
+
+/* H += scale * X^T X over n calibration tokens  (dingiv.github.io page,
+ * section GPTQ: H = 2 X X^T, so scale = 2 for that definition).
+ *  H      fp32, d x d row-major (leading dimension d), accumulated in place:
+ *         the caller zeroes it before the first chunk.  Only the upper
+ *         triangle including the diagonal (H[i][j], i <= j) is written; the
+ *         strict lower triangle is never touched.
+ *  X      bf16 token-major activations, n rows of d values, row stride ldx
+ *         elements (ldx >= d, ldx % 8 == 0, X 16-byte aligned).  This is
+ *         X^T of the page's d x n matrix, the layout a model's activations
+ *         have.  Chunks of any size may be accumulated by repeated calls.
+ *  d      % 8 == 0, 8 <= d <= 65536.   n >= 0 (n == 0 is a no-op).
+ * Summation order over tokens within one call is not fixed (split over
+ * tokens with fp32 atomic adds), so results may differ in the last bits
+ * between runs.  Asynchronous. */
+gptq_status gptq_hessian_accumulate(float* H, const void* X, int64_t n,
+                                    int64_t d, int64_t ldx, float scale,
+                                    void* stream);
+
+/* From H (upper triangle, as left by gptq_hessian_accumulate) compute the
+ * damped H' = H + lambda I, lambda = damp_rel * mean(diag H), with a dead
+ * input channel (H_ii == 0) given H'_ii = 1 and flagged in dead_mask, and
+ * then G = the upper triangular U with U^T U = H'^-1 (dingiv.github.io page,
+ * section GPTQ: the Cholesky factor of H^-1 through which all updates go).
+ * Computed in fp64 as U = V^-1 where H' = V V^T with V upper triangular
+ * (a Cholesky factorisation taken from the last row upward).
+ *  H          fp32 d x d, read-only; only the upper triangle is read.
+ *  G          fp32 d x d output; upper triangle = U, strict lower = 0.
+ *  dead_mask  uint8[d] output, 1 for a dead channel.
+ *  bad_pivot  host int64 out (may be NULL): -1, or the first column (in the
+ *             original order) whose pivot was not positive and finite.
+ *  ws         workspace of at least gptq_workspace_size(?, d, cfg) bytes.
+ * Returns GPTQ_ERR_NOT_SPD if a pivot fails, GPTQ_ERR_NONFINITE if H has a
+ * NaN/Inf on its diagonal.  Synchronizes `stream` once. */
+gptq_status gptq_prepare_hinv(const float* H, int64_t d, double damp_rel,
+                              float* G, uint8_t* dead_mask,
+                              void* ws, size_t ws_bytes,
+                              int64_t* bad_pivot, void* stream);
+
+/* Quantize W column by column, left to right, in blocks of cfg->block
+ * columns (dingiv.github.io page, section GPTQ, and its three refinements:
+ * fixed order, Cholesky factor, lazy batched updates):
+ *   for column q: code it, e = (w_q - w^_q) / G_qq, subtract e * G[q][k]
+ *   from every later column k of the block at once; after the block,
+ *   W[:, right] -= E * G[block, right].
+ *  W          fp32 d_row x d_col input weights, read-only (a working copy
+ *             is kept in the workspace).  Columns flagged in dead_mask are
+ *             zeroed before quantization.
+ *  G          fp32 d_col x d_col from gptq_prepare_hinv (upper triangle read).
+ *  dead_mask  uint8[d_col] or NULL (no dead channels).
+ *  qweight    uint32 d_row x (d_col*bits/32) output: row r's codes as a
+ *             little-endian bit stream, code k at bits [bits*k, bits*k+bits),
+ *             word w holding bits [32w, 32w+32).
+ *  scales     fp32 d_row x n_groups output (n_groups = 1 when group_size is
+ *             0, else d_col / group_size), row-major.
+ *  zeros      uint8 d_row x n_groups output (integer zero points).
+ *  Shapes: d_row >= 1, d_col % 32 == 0, d_col >= 32.  Asynchronous. */
+gptq_status gptq_quantize_layer(const float* W, int64_t d_row, int64_t d_col,
+                                const float* G, const uint8_t* dead_mask,
+                                const gptq_config* cfg, uint32_t* qweight,
+                                float* scales, uint8_t* zeros,
+                                void* ws, size_t ws_bytes, void* stream);
+
+/* Dequantize the packed output and measure the layer loss of the page's
+ * objective through the Hessian: loss = 1/2 * sum_r dW_r H dW_r^T with
+ * dW = W - W^, which equals ||W X - W^ X||_F^2 for H = 2 X X^T
+ * (dingiv.github.io page, section GPTQ, the per-layer objective).
+ *  qweight, scales, zeros  as written by gptq_quantize_layer.
+ *  W       fp32 d_row x d_col, the original weights.
+ *  H       fp32 d_col x d_col, the UNdamped Hessian (upper triangle read).
+ *  W_hat   fp32 d_row x d_col output of dequantized weights, or NULL.
+ *  loss    host double out (may be NULL).
+ * Synchronizes `stream` once. */
+gptq_status gptq_dequant_check(const uint32_t* qweight, const float* scales,
+                               const uint8_t* zeros, const float* W,
+                               const float* H, int64_t d_row, int64_t d_col,
+                               const gptq_config* cfg, float* W_hat,
+                               double* loss, void* ws, size_t ws_bytes,
+                               void* stream);
+
+/* Synchronize `stream`, then return and clear the device status word that
+ * kernels set when a bounded internal wait runs out (GPTQ_ERR_TIMEOUT). */
+gptq_status gptq_device_status(void* stream);
+
+/* Number of kernels this library has launched in this process (all devices,
+ * all streams).  Instrumentation for benchmarks: the difference across a
+ * timed region is the launch count of that region.  The paper has no
+ * counterpart; it is not part of the method. */
+uint64_t gptq_launch_count(void);
+
+/* Static, human-readable name of a status code. */
+const char* gptq_status_string(gptq_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GPTQ_B200_H */

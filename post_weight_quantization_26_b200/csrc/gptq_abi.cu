@@ -1,0 +1,531 @@
+// extern "C" entry points of libgptq.so (declared in include/gptq.h): argument
+// validation, workspace layout, TMA descriptor encoding and the launch
+// sequences of the GPTQ stages.  All device kernels are in the .cuh files
+// included below, compiled as one translation unit.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/gptq.h"
+#include "chol_fp64.cuh"
+#include "common.cuh"
+#include "quantize.cuh"
+#include "syrk_tcgen05.cuh"
+
+namespace {
+
+using namespace gptq;
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+inline bool aligned(const void* p, size_t a) {
+  return (reinterpret_cast<uintptr_t>(p) % a) == 0;
+}
+
+#define GPTQ_CUDA_TRY(expr)                          \
+  do {                                               \
+    cudaError_t e_ = (expr);                         \
+    if (e_ != cudaSuccess) {                         \
+      std::fprintf(stderr, "gptq: %s failed: %s\n", #expr, cudaGetErrorString(e_)); \
+      return GPTQ_ERR_CUDA;                          \
+    }                                                \
+  } while (0)
+
+std::atomic<uint64_t> g_launches{0};
+
+#define GPTQ_LAUNCH_CHECK()                          \
+  do {                                               \
+    g_launches.fetch_add(1, std::memory_order_relaxed); \
+    cudaError_t e_ = cudaGetLastError();             \
+    if (e_ != cudaSuccess) {                         \
+      std::fprintf(stderr, "gptq: launch failed at %s:%d: %s\n", __FILE__, __LINE__, \
+                   cudaGetErrorString(e_));          \
+      return GPTQ_ERR_CUDA;                          \
+    }                                                \
+  } while (0)
+
+// ------------------------------------------------------------ device setup
+struct DeviceInfo {
+  bool ready = false;
+  int num_sms = 0;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[64];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+gptq_status device_setup(int* num_sms) {
+  int dev = 0;
+  GPTQ_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return GPTQ_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& di = g_dev[dev];
+  if (!di.ready) {
+    GPTQ_CUDA_TRY(cudaDeviceGetAttribute(&di.num_sms, cudaDevAttrMultiProcessorCount, dev));
+    GPTQ_CUDA_TRY(cudaFuncSetAttribute(syrk::syrk_bf16_tcgen05_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       syrk::SMEM_BYTES));
+    GPTQ_CUDA_TRY(cudaFuncSetAttribute(chol::dgemm_grouped_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       chol::GEMM_SMEM));
+    GPTQ_CUDA_TRY(cudaFuncSetAttribute(chol::leaf_potrf_inv_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       chol::LEAF_SMEM));
+    GPTQ_CUDA_TRY(cudaFuncSetAttribute(quant::block_quant_kernel<128, 0>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       quant::block_quant_smem<128>()));
+    GPTQ_CUDA_TRY(cudaFuncSetAttribute(quant::block_quant_kernel<128, 32>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       quant::block_quant_smem<128>()));
+    GPTQ_CUDA_TRY(cudaFuncSetAttribute(quant::block_quant_kernel<128, 64>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       quant::block_quant_smem<128>()));
+    GPTQ_CUDA_TRY(cudaFuncSetAttribute(quant::block_quant_kernel<64, 0>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       quant::block_quant_smem<64>()));
+    GPTQ_CUDA_TRY(cudaFuncSetAttribute(quant::block_quant_kernel<64, 32>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       quant::block_quant_smem<64>()));
+    if (!g_encode) {
+      cudaDriverEntryPointQueryResult q;
+      void* fn = nullptr;
+      GPTQ_CUDA_TRY(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q));
+      if (q != cudaDriverEntryPointSuccess || !fn) return GPTQ_ERR_CUDA;
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    di.ready = true;
+  }
+  if (num_sms) *num_sms = di.num_sms;
+  return GPTQ_OK;
+}
+
+bool config_ok(const gptq_config* c, int64_t d_col) {
+  if (!c) return false;
+  if (c->bits < 2 || c->bits > 4) return false;
+  if (c->block != 32 && c->block != 64 && c->block != 128) return false;
+  if (c->sym != 0 && c->sym != 1) return false;
+  if (!(c->damp_rel >= 0.0) || !std::isfinite(c->damp_rel)) return false;
+  const int g = c->group_size;
+  if (g < 0) return false;
+  if (g > 0) {
+    if (g % 32 != 0) return false;
+    if (d_col % g != 0) return false;
+    if (!(c->block % g == 0 || g % c->block == 0)) return false;
+  }
+  return true;
+}
+
+// ---------------------------------------------------------- workspace map
+struct PrepareWs {
+  size_t stats, istat, pivot, A, Xd, total;
+};
+PrepareWs prepare_layout(int64_t d) {
+  PrepareWs w{};
+  size_t off = 0;
+  w.stats = off; off = align_up(off + 8);
+  w.istat = off; off = align_up(off + 8);
+  w.pivot = off; off = align_up(off + 8);
+  w.A = off; off = align_up(off + static_cast<size_t>(d) * d * 8);
+  const int64_t nt = (d + chol::NB - 1) / chol::NB;
+  w.Xd = off; off = align_up(off + static_cast<size_t>(nt) * chol::NB * chol::NB * 8);
+  w.total = off;
+  return w;
+}
+
+struct QuantWs {
+  size_t Wk, E, total;
+};
+QuantWs quant_layout(int64_t d_row, int64_t d_col, int block) {
+  QuantWs w{};
+  size_t off = 0;
+  w.Wk = off; off = align_up(off + static_cast<size_t>(d_row) * d_col * 4);
+  w.E = off; off = align_up(off + static_cast<size_t>(d_row) * block * 4);
+  w.total = off;
+  return w;
+}
+
+struct CheckWs {
+  size_t partials, loss, total;
+};
+CheckWs check_layout(int64_t d_row, int64_t d_col) {
+  CheckWs w{};
+  const size_t tiles = static_cast<size_t>((d_row + 127) / 128) * ((d_col + 127) / 128);
+  size_t off = 0;
+  w.partials = off; off = align_up(off + tiles * 8);
+  w.loss = off; off = align_up(off + 8);
+  w.total = off;
+  return w;
+}
+
+// --------------------------------------------------------- SYRK launching
+void choose_split(int ntiles, int n, int num_sms, int* split_tokens, int* nsplit) {
+  const int nkb = (n + syrk::BK - 1) / syrk::BK;
+  double best = 1e300;
+  int best_s = 1;
+  const int max_s = std::max(1, std::min(64, nkb));
+  for (int s = 1; s <= max_s; ++s) {
+    const int kb_per = (nkb + s - 1) / s;
+    const int s_eff = (nkb + kb_per - 1) / kb_per;
+    const long long units = static_cast<long long>(ntiles) * s_eff;
+    const long long waves = (units + num_sms - 1) / num_sms;
+    // a unit costs its k-stages plus a fixed ramp/epilogue share
+    const double cost = static_cast<double>(waves) * (kb_per + 6);
+    if (cost < best * 0.999) { best = cost; best_s = s; }
+  }
+  const int kb_per = (nkb + best_s - 1) / best_s;
+  *split_tokens = kb_per * syrk::BK;
+  *nsplit = (nkb + kb_per - 1) / kb_per;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* gptq_status_string(gptq_status s) {
+  switch (s) {
+    case GPTQ_OK: return "GPTQ_OK";
+    case GPTQ_ERR_INVALID: return "GPTQ_ERR_INVALID";
+    case GPTQ_ERR_NOT_SPD: return "GPTQ_ERR_NOT_SPD";
+    case GPTQ_ERR_NONFINITE: return "GPTQ_ERR_NONFINITE";
+    case GPTQ_ERR_WORKSPACE: return "GPTQ_ERR_WORKSPACE";
+    case GPTQ_ERR_CUDA: return "GPTQ_ERR_CUDA";
+    case GPTQ_ERR_TIMEOUT: return "GPTQ_ERR_TIMEOUT";
+  }
+  return "GPTQ_ERR_UNKNOWN";
+}
+
+uint64_t gptq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+size_t gptq_workspace_size(int64_t d_row, int64_t d_col, const gptq_config* cfg) {
+  if (d_row < 1 || d_col < 32 || d_col % 32 != 0 || d_col > 65536 || !config_ok(cfg, d_col))
+    return 0;
+  const size_t a = prepare_layout(d_col).total;
+  const size_t b = quant_layout(d_row, d_col, cfg->block).total;
+  const size_t c = check_layout(d_row, d_col).total;
+  return std::max(a, std::max(b, c));
+}
+
+gptq_status gptq_device_status(void* stream) {
+  GPTQ_CUDA_TRY(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  int v = 0, zero = 0;
+  GPTQ_CUDA_TRY(cudaMemcpyFromSymbol(&v, gptq::g_device_status, sizeof(int)));
+  GPTQ_CUDA_TRY(cudaMemcpyToSymbol(gptq::g_device_status, &zero, sizeof(int)));
+  return static_cast<gptq_status>(v);
+}
+
+gptq_status gptq_hessian_accumulate(float* H, const void* X, int64_t n, int64_t d, int64_t ldx,
+                                    float scale, void* stream) {
+  if (!H || !X) return GPTQ_ERR_INVALID;
+  if (d < 8 || d > 65536 || d % 8 != 0) return GPTQ_ERR_INVALID;
+  if (n < 0 || n > (int64_t(1) << 31) - 1) return GPTQ_ERR_INVALID;
+  if (ldx < d || ldx % 8 != 0) return GPTQ_ERR_INVALID;
+  if (!aligned(X, 16) || !aligned(H, 16)) return GPTQ_ERR_INVALID;
+  if (!std::isfinite(scale)) return GPTQ_ERR_INVALID;
+  if (n == 0) return GPTQ_OK;
+  int num_sms = 0;
+  gptq_status st = device_setup(&num_sms);
+  if (st != GPTQ_OK) return st;
+
+  CUtensorMap tmap;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ldx) * 2};
+  const cuuint32_t box[2] = {syrk::BOX, syrk::BK};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult cr = g_encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(X), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) {
+    std::fprintf(stderr, "gptq: cuTensorMapEncodeTiled failed (%d)\n", static_cast<int>(cr));
+    return GPTQ_ERR_CUDA;
+  }
+
+  syrk::Params p{};
+  p.H = H;
+  p.d = static_cast<int>(d);
+  p.n = static_cast<int>(n);
+  p.scale = scale;
+  p.nti = static_cast<int>((d + syrk::BM - 1) / syrk::BM);
+  p.ntj = static_cast<int>((d + syrk::BN - 1) / syrk::BN);
+  {
+    const int h = p.nti >> 1;
+    p.ntiles = p.nti * p.ntj - (h * (h - 1) + (p.nti & 1) * h);
+  }
+  choose_split(p.ntiles, p.n, num_sms, &p.split_tokens, &p.nsplit);
+  p.units = p.ntiles * p.nsplit;
+  const int grid = std::min(p.units, num_sms);
+  syrk::syrk_bf16_tcgen05_kernel<<<grid, syrk::NUM_THREADS, syrk::SMEM_BYTES,
+                                   static_cast<cudaStream_t>(stream)>>>(tmap, p);
+  GPTQ_LAUNCH_CHECK();
+  return GPTQ_OK;
+}
+
+namespace {
+
+gptq_status launch_gemm_batch(std::vector<chol::GemmProblem>& probs, cudaStream_t s) {
+  size_t i = 0;
+  while (i < probs.size()) {
+    chol::GemmBatch b{};
+    int tiles = 0;
+    b.count = 0;
+    while (i < probs.size() && b.count < chol::MAXP) {
+      const chol::GemmProblem& q = probs[i];
+      const int tm = (q.M + chol::TM - 1) / chol::TM, tn = (q.N + chol::TN - 1) / chol::TN;
+      const int nt = q.lower_only ? tm * (tm + 1) / 2 : tm * tn;
+      if (q.M > 0 && q.N > 0) {
+        b.tile_start[b.count] = tiles;
+        b.p[b.count] = q;
+        tiles += nt;
+        ++b.count;
+      }
+      ++i;
+    }
+    b.tile_start[b.count] = tiles;
+    if (tiles > 0) {
+      chol::dgemm_grouped_kernel<<<tiles, chol::GEMM_THREADS, chol::GEMM_SMEM, s>>>(b);
+      GPTQ_LAUNCH_CHECK();
+    }
+  }
+  return GPTQ_OK;
+}
+
+struct Node {
+  int a, m, b, height;
+};
+
+int build_tree(int a, int b, std::vector<Node>& out) {
+  // nodes over [a, b) in units of NB blocks (a, b are block indices)
+  if (b - a <= 1) return 0;
+  const int m = a + (b - a + 1) / 2;
+  const int hl = build_tree(a, m, out);
+  const int hr = build_tree(m, b, out);
+  const int h = 1 + std::max(hl, hr);
+  out.push_back(Node{a, m, b, h});
+  return h;
+}
+
+}  // namespace
+
+gptq_status gptq_prepare_hinv(const float* H, int64_t d, double damp_rel, float* G,
+                              uint8_t* dead_mask, void* ws, size_t ws_bytes,
+                              int64_t* bad_pivot, void* stream) {
+  if (bad_pivot) *bad_pivot = -1;
+  if (!H || !G || !dead_mask) return GPTQ_ERR_INVALID;
+  if (d < 8 || d > 65536 || d % 8 != 0) return GPTQ_ERR_INVALID;
+  if (!(damp_rel >= 0.0) || !std::isfinite(damp_rel)) return GPTQ_ERR_INVALID;
+  const PrepareWs L = prepare_layout(d);
+  if (!ws || !aligned(ws, kAlign) || ws_bytes < L.total) return GPTQ_ERR_WORKSPACE;
+  gptq_status st = device_setup(nullptr);
+  if (st != GPTQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  double* stats = reinterpret_cast<double*>(base + L.stats);
+  int* istat = reinterpret_cast<int*>(base + L.istat);
+  long long* pivot = reinterpret_cast<long long*>(base + L.pivot);
+  double* A = reinterpret_cast<double*>(base + L.A);
+  double* Xd = reinterpret_cast<double*>(base + L.Xd);
+  const int di = static_cast<int>(d);
+  const int nt = (di + chol::NB - 1) / chol::NB;
+
+  GPTQ_CUDA_TRY(cudaMemsetAsync(pivot, 0xFF, 8, s));
+  chol::diag_stats_kernel<<<1, 1024, 0, s>>>(H, di, damp_rel, dead_mask, stats, istat);
+  GPTQ_LAUNCH_CHECK();
+  {
+    dim3 grid((di + 255) / 256, di);
+    chol::reverse_damp_fill_kernel<<<grid, 256, 0, s>>>(H, di, stats, A);
+    GPTQ_LAUNCH_CHECK();
+  }
+  // blocked right-looking Cholesky of A (the reversed, damped H)
+  for (int k = 0; k < nt; ++k) {
+    const int k0 = k * chol::NB;
+    const int nk = std::min(chol::NB, di - k0);
+    double* Xk = Xd + static_cast<size_t>(k) * chol::NB * chol::NB;
+    chol::leaf_potrf_inv_kernel<<<1, chol::LEAF_THREADS, chol::LEAF_SMEM, s>>>(A, di, k0, nk, Xk,
+                                                                                 pivot);
+    GPTQ_LAUNCH_CHECK();
+    const int rest = di - k0 - nk;
+    if (rest <= 0) continue;
+    std::vector<chol::GemmProblem> v(1);
+    chol::GemmProblem& pn = v[0];
+    pn = chol::GemmProblem{};
+    pn.A = A + static_cast<size_t>(k0 + nk) * di + k0;
+    pn.lda = di;
+    pn.a_trans = 0;
+    pn.B = Xk;
+    pn.ldb = chol::NB;
+    pn.b_trans = 1;
+    pn.C = A + static_cast<size_t>(k0 + nk) * di + k0;
+    pn.ldc = di;
+    pn.M = rest; pn.N = nk; pn.K = nk;
+    pn.alpha = 1.0; pn.beta = 0.0;
+    st = launch_gemm_batch(v, s);
+    if (st != GPTQ_OK) return st;
+    chol::GemmProblem up{};
+    up.A = A + static_cast<size_t>(k0 + nk) * di + k0;
+    up.lda = di;
+    up.a_trans = 0;
+    up.B = A + static_cast<size_t>(k0 + nk) * di + k0;
+    up.ldb = di;
+    up.b_trans = 1;
+    up.C = A + static_cast<size_t>(k0 + nk) * di + (k0 + nk);
+    up.ldc = di;
+    up.M = rest; up.N = rest; up.K = nk;
+    up.lower_only = 1;
+    up.alpha = -1.0; up.beta = 1.0;
+    v[0] = up;
+    st = launch_gemm_batch(v, s);
+    if (st != GPTQ_OK) return st;
+  }
+  // triangular inverse: diagonal blocks from the leaves, then by tree height
+  chol::place_diag_inverses_kernel<<<nt, 256, 0, s>>>(A, di, Xd);
+  GPTQ_LAUNCH_CHECK();
+  std::vector<Node> nodes;
+  const int height = build_tree(0, nt, nodes);
+  for (int h = 1; h <= height; ++h) {
+    std::vector<chol::GemmProblem> g1, g2;
+    for (const Node& nd : nodes) {
+      if (nd.height != h) continue;
+      const int a = nd.a * chol::NB, m = nd.m * chol::NB, b = std::min(nd.b * chol::NB, di);
+      chol::GemmProblem p1{};  // T^T = X11^T L21^T stored at A[a:m, m:b]
+      p1.A = A + static_cast<size_t>(a) * di + a; p1.lda = di; p1.a_trans = 1; p1.kmode = 2;
+      p1.B = A + static_cast<size_t>(m) * di + a; p1.ldb = di; p1.b_trans = 1;
+      p1.C = A + static_cast<size_t>(a) * di + m; p1.ldc = di;
+      p1.M = m - a; p1.N = b - m; p1.K = m - a;
+      p1.alpha = 1.0; p1.beta = 0.0;
+      g1.push_back(p1);
+      chol::GemmProblem p2{};  // X21 = -X22 T
+      p2.A = A + static_cast<size_t>(m) * di + m; p2.lda = di; p2.a_trans = 0; p2.kmode = 1;
+      p2.B = A + static_cast<size_t>(a) * di + m; p2.ldb = di; p2.b_trans = 1;
+      p2.C = A + static_cast<size_t>(m) * di + a; p2.ldc = di;
+      p2.M = b - m; p2.N = m - a; p2.K = b - m;
+      p2.alpha = -1.0; p2.beta = 0.0;
+      g2.push_back(p2);
+    }
+    st = launch_gemm_batch(g1, s);
+    if (st != GPTQ_OK) return st;
+    st = launch_gemm_batch(g2, s);
+    if (st != GPTQ_OK) return st;
+  }
+  {
+    dim3 grid((di + 255) / 256, di);
+    chol::write_g_kernel<<<grid, 256, 0, s>>>(A, di, G);
+    GPTQ_LAUNCH_CHECK();
+  }
+  long long host_pivot = -1;
+  int host_istat = 0;
+  GPTQ_CUDA_TRY(cudaMemcpyAsync(&host_pivot, pivot, 8, cudaMemcpyDeviceToHost, s));
+  GPTQ_CUDA_TRY(cudaMemcpyAsync(&host_istat, istat, 4, cudaMemcpyDeviceToHost, s));
+  GPTQ_CUDA_TRY(cudaStreamSynchronize(s));
+  if (bad_pivot) *bad_pivot = host_pivot;
+  if (host_istat) return GPTQ_ERR_NONFINITE;
+  if (host_pivot >= 0) return GPTQ_ERR_NOT_SPD;
+  return GPTQ_OK;
+}
+
+gptq_status gptq_quantize_layer(const float* W, int64_t d_row, int64_t d_col, const float* G,
+                                const uint8_t* dead_mask, const gptq_config* cfg,
+                                uint32_t* qweight, float* scales, uint8_t* zeros, void* ws,
+                                size_t ws_bytes, void* stream) {
+  if (!W || !G || !qweight || !scales || !zeros) return GPTQ_ERR_INVALID;
+  if (d_row < 1 || d_row > (int64_t(1) << 24) || d_col < 32 || d_col % 32 != 0 ||
+      d_col > 65536)
+    return GPTQ_ERR_INVALID;
+  if (!config_ok(cfg, d_col)) return GPTQ_ERR_INVALID;
+  if (!aligned(W, 16) || !aligned(G, 16) || !aligned(qweight, 4) || !aligned(scales, 4))
+    return GPTQ_ERR_INVALID;
+  if (dead_mask && !aligned(dead_mask, 4)) return GPTQ_ERR_INVALID;
+  const QuantWs L = quant_layout(d_row, d_col, cfg->block);
+  if (!ws || !aligned(ws, kAlign) || ws_bytes < L.total) return GPTQ_ERR_WORKSPACE;
+  gptq_status st = device_setup(nullptr);
+  if (st != GPTQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  float* Wk = reinterpret_cast<float*>(base + L.Wk);
+  float* E = reinterpret_cast<float*>(base + L.E);
+  const int dr = static_cast<int>(d_row), dc = static_cast<int>(d_col);
+  const int B = cfg->block, g = cfg->group_size;
+  const int n_groups = g ? dc / g : 1;
+  const int per_channel = g == 0;
+
+  quant::prepare_rows_kernel<<<(dr + 7) / 8, 256, 0, s>>>(W, Wk, dead_mask, dr, dc, cfg->bits,
+                                                           cfg->sym, per_channel, scales, zeros);
+  GPTQ_LAUNCH_CHECK();
+  const int gs_inblock = (g > 0 && g < B) ? g : 0;
+  const dim3 qgrid((dr + quant::QROWS - 1) / quant::QROWS);
+  for (int j0 = 0; j0 < dc; j0 += B) {
+    const int ncols = std::min(B, dc - j0);
+#define GPTQ_BQ(BB, GSV)                                                                     \
+  quant::block_quant_kernel<BB, GSV><<<qgrid, quant::QTHREADS, quant::block_quant_smem<BB>(), s>>>( \
+      Wk, dr, dc, j0, ncols, G, E, qweight, scales, zeros, cfg->bits, cfg->sym, g, n_groups,   \
+      per_channel)
+    if (B == 128 && gs_inblock == 0) GPTQ_BQ(128, 0);
+    else if (B == 128 && gs_inblock == 32) GPTQ_BQ(128, 32);
+    else if (B == 128 && gs_inblock == 64) GPTQ_BQ(128, 64);
+    else if (B == 64 && gs_inblock == 0) GPTQ_BQ(64, 0);
+    else if (B == 64 && gs_inblock == 32) GPTQ_BQ(64, 32);
+    else if (B == 32) GPTQ_BQ(32, 0);
+    else return GPTQ_ERR_INVALID;
+#undef GPTQ_BQ
+    GPTQ_LAUNCH_CHECK();
+    const int j1 = j0 + ncols;
+    if (j1 < dc) {
+      const int N = dc - j1;
+      const dim3 ugrid((dr + quant::UT - 1) / quant::UT, (N + quant::UT - 1) / quant::UT);
+      quant::trailing_update_kernel<<<ugrid, quant::UTHREADS, 0, s>>>(
+          Wk + j1, E, G + static_cast<size_t>(j0) * dc + j1, dr, N, B, dc, dc);
+      GPTQ_LAUNCH_CHECK();
+    }
+  }
+  return GPTQ_OK;
+}
+
+gptq_status gptq_dequant_check(const uint32_t* qweight, const float* scales, const uint8_t* zeros,
+                               const float* W, const float* H, int64_t d_row, int64_t d_col,
+                               const gptq_config* cfg, float* W_hat, double* loss, void* ws,
+                               size_t ws_bytes, void* stream) {
+  if (!qweight || !scales || !zeros) return GPTQ_ERR_INVALID;
+  if (d_row < 1 || d_row > (int64_t(1) << 24) || d_col < 32 || d_col % 32 != 0 ||
+      d_col > 65536)
+    return GPTQ_ERR_INVALID;
+  if (!config_ok(cfg, d_col)) return GPTQ_ERR_INVALID;
+  if (loss && (!W || !H)) return GPTQ_ERR_INVALID;
+  const CheckWs L = check_layout(d_row, d_col);
+  if (loss && (!ws || !aligned(ws, kAlign) || ws_bytes < L.total)) return GPTQ_ERR_WORKSPACE;
+  gptq_status st = device_setup(nullptr);
+  if (st != GPTQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int dr = static_cast<int>(d_row), dc = static_cast<int>(d_col);
+  const int g = cfg->group_size;
+  const int n_groups = g ? dc / g : 1;
+  if (W_hat) {
+    quant::dequant_kernel<<<1184, 256, 0, s>>>(qweight, scales, zeros, dr, dc, cfg->bits, g,
+                                               n_groups, W_hat);
+    GPTQ_LAUNCH_CHECK();
+  }
+  if (loss) {
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    double* partials = reinterpret_cast<double*>(base + L.partials);
+    double* dloss = reinterpret_cast<double*>(base + L.loss);
+    const dim3 grid((dr + 127) / 128, (dc + 127) / 128);
+    quant::loss_tiles_kernel<<<grid, 256, 0, s>>>(qweight, scales, zeros, W, H, dr, dc,
+                                                  cfg->bits, g, n_groups, partials);
+    GPTQ_LAUNCH_CHECK();
+    quant::sum_partials_kernel<<<1, 1024, 0, s>>>(partials, static_cast<int>(grid.x * grid.y),
+                                                  dloss);
+    GPTQ_LAUNCH_CHECK();
+    GPTQ_CUDA_TRY(cudaMemcpyAsync(loss, dloss, 8, cudaMemcpyDeviceToHost, s));
+  }
+  GPTQ_CUDA_TRY(cudaStreamSynchronize(s));
+  return GPTQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,231 @@
+// Hessian accumulation H += scale * X^T X on the 5th-generation tensor cores.
+//
+// dingiv.github.io "量化" page, section GPTQ: H = 2 X X^T over the
+// calibration tokens.  X arrives token-major (n rows of d bf16 values), so
+// with K = tokens both MMA operands are "MN-major": A(m,k) = X[k][i0+m] and
+// B(n,k) = X[k][j0+n] come from the same tensor.  Only tiles that touch the
+// upper triangle (i <= j) are computed, 128 x 256 per tile, and tokens are
+// split into S chunks so that tiles x chunks fill the 148 SMs evenly; the
+// chunk partials meet in H through fp32 vector atomic adds.
+//
+// Warp roles (192 threads, one CTA per SM, persistent over work units):
+//   warp 0      TMA producer: 64-token stages, A = 2 boxes of 64 features,
+//               B = 4 boxes, 128-byte swizzle, STAGES-deep ring.
+//   warp 1      allocates 512 TMEM columns (two 128x256 fp32 accumulators)
+//               and issues tcgen05.mma (one thread), K = 16 per instruction.
+//   warps 2..5  epilogue: tcgen05.ld the accumulator (each warp its 32-lane
+//               quarter), scale, mask to the upper triangle, atomically add.
+// The accumulator is double-buffered so the epilogue of one unit overlaps
+// the MMAs of the next.  Every mbarrier wait is bounded.
+#pragma once
+
+#include "common.cuh"
+
+namespace gptq {
+namespace syrk {
+
+constexpr int BM = 128;     // rows of H per tile (features i)
+constexpr int BN = 256;     // columns of H per tile (features j)
+constexpr int BK = 64;      // tokens per pipeline stage
+constexpr int STAGES = 4;
+constexpr int BOX = 64;     // TMA box: 64 features (128 B) x 64 tokens
+constexpr int BOX_BYTES = BOX * BK * 2;               // 8 KB
+constexpr int A_BYTES = BM * BK * 2;                  // 16 KB
+constexpr int B_BYTES = BN * BK * 2;                  // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;        // 48 KB
+constexpr int NUM_THREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+
+// Instruction descriptor, kind::f16: fp32 accumulate (bits 4-5 = 1), A and B
+// bf16 (bits 7-9 = 1, 10-12 = 1), both MN-major (bits 15, 16), N>>3 at
+// bits 17-22, M>>4 at bits 24-28.
+constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
+                           (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
+
+struct Params {
+  float* H;
+  int d;
+  int n;
+  float scale;
+  int nti;        // row tiles: ceil(d / BM)
+  int ntj;        // column tiles: ceil(d / BN)
+  int ntiles;     // tiles touching the upper triangle
+  int split_tokens;  // tokens per chunk (multiple of BK)
+  int nsplit;
+  int units;      // ntiles * nsplit
+};
+
+// Tiles of row-tile ti that touch the upper triangle start at column tile
+// floor(ti / 2) (since BN = 2 BM); prefix(ti) = number of tiles before row ti.
+__device__ __forceinline__ int tiles_before(int ti, int ntj) {
+  const int h = ti >> 1;
+  return ti * ntj - (h * (h - 1) + (ti & 1) * h);
+}
+
+__device__ __forceinline__ void decode_unit(const Params& p, int u, int& ti, int& tj,
+                                            int& k0, int& nk) {
+  const int s = u / p.ntiles;
+  const int t = u - s * p.ntiles;
+  int lo = 0, hi = p.nti - 1;  // largest ti with tiles_before(ti) <= t
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (tiles_before(mid, p.ntj) <= t) lo = mid; else hi = mid - 1;
+  }
+  ti = lo;
+  tj = (ti >> 1) + (t - tiles_before(ti, p.ntj));
+  k0 = s * p.split_tokens;
+  const int k1 = min(p.n, k0 + p.split_tokens);
+  nk = (k1 - k0 + BK - 1) / BK;
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+syrk_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-byte aligned ring of stages (128B-swizzle atoms are 1024 B).
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t ring = (raw + 1023u) & ~1023u;
+  uint8_t* ring_ptr = smem_raw + (ring - raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring_ptr + STAGES * STAGE_BYTES);
+  // bars[0..S) full, [S..2S) empty, [2S..2S+2) tmem_full, [2S+2..2S+4) tmem_empty
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = full0 + 8u * STAGES;
+  const uint32_t tfull0 = full0 + 16u * STAGES;
+  const uint32_t tempty0 = tfull0 + 16u;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full0 + 8u * s, 1);
+      mbar_init(empty0 + 8u * s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull0 + 8u * a, 1);
+      mbar_init(tempty0 + 8u * a, 4);  // one arrive per epilogue warp
+    }
+    *abort_flag = 0;
+    mbar_fence_init();
+    tma_prefetch_desc(&tmap_x);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+        int ti, tj, k0, nk;
+        decode_unit(p, u, ti, tj, k0, nk);
+        for (int kt = 0; kt < nk; ++kt) {
+          if (!mbar_wait_bounded(empty0 + 8u * stage, phase ^ 1u, abort_flag)) { ok = false; break; }
+          const uint32_t fb = full0 + 8u * stage;
+          mbar_arrive_expect_tx(fb, STAGE_BYTES);
+          const uint32_t sa = ring + stage * STAGE_BYTES;
+          const uint32_t sb = sa + A_BYTES;
+          const int tok = k0 + kt * BK;
+#pragma unroll
+          for (int c = 0; c < BM / BOX; ++c) tma_load_2d(sa + c * BOX_BYTES, &tmap_x, fb, ti * BM + c * BOX, tok);
+#pragma unroll
+          for (int c = 0; c < BN / BOX; ++c) tma_load_2d(sb + c * BOX_BYTES, &tmap_x, fb, tj * BN + c * BOX, tok);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------------- MMA
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      int lu = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x, ++lu) {
+        int ti, tj, k0, nk;
+        decode_unit(p, u, ti, tj, k0, nk);
+        const uint32_t acc = lu & 1;
+        if (!mbar_wait_bounded(tempty0 + 8u * acc, ((lu >> 1) & 1) ^ 1u, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kt = 0; kt < nk; ++kt) {
+          if (!mbar_wait_bounded(full0 + 8u * stage, phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = ring + stage * STAGE_BYTES;
+          const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            // 16 tokens = two 8-row core groups of 128 B each = 2048 B.
+            const uint64_t ad = smem_desc_sw128(sa + kk * 2048, BOX_BYTES, 1024);
+            const uint64_t bd = smem_desc_sw128(sb + kk * 2048, BOX_BYTES, 1024);
+            mma_f16_ss(d_tmem, ad, bd, IDESC, (kt | kk) != 0);
+          }
+          mma_commit(empty0 + 8u * stage);  // frees the stage when these MMAs finish
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        mma_commit(tfull0 + 8u * acc);  // accumulator ready for the epilogue
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter+32)
+    int lu = 0;
+    for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++lu) {
+      int ti, tj, k0, nk;
+      decode_unit(p, u, ti, tj, k0, nk);
+      const uint32_t acc = lu & 1;
+      if (!mbar_wait_bounded(tfull0 + 8u * acc, (lu >> 1) & 1, abort_flag)) break;
+      tc_fence_after();
+      const int row = ti * BM + quarter * 32 + lane;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
+      float* hrow = p.H + static_cast<size_t>(row) * p.d;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(t_row + c * 32, r);
+        tmem_ld_wait();
+        const int jb = tj * BN + c * 32;
+        if (row < p.d && jb + 31 >= row && jb < p.d) {
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            const int j = jb + 4 * v;
+            if (j >= p.d || j + 3 < row) continue;
+            float4 val = make_float4(__uint_as_float(r[4 * v]) * p.scale,
+                                     __uint_as_float(r[4 * v + 1]) * p.scale,
+                                     __uint_as_float(r[4 * v + 2]) * p.scale,
+                                     __uint_as_float(r[4 * v + 3]) * p.scale);
+            if (j >= row) {
+              atomicAdd(reinterpret_cast<float4*>(hrow + j), val);
+            } else {  // the 4-vector straddles the diagonal
+              if (j + 1 >= row) atomicAdd(hrow + j + 1, val.y);
+              if (j + 2 >= row) atomicAdd(hrow + j + 2, val.z);
+              atomicAdd(hrow + j + 3, val.w);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty0 + 8u * acc);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace syrk
+}  // namespace gptq
