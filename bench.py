@@ -39,10 +39,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
 def parse_args():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=5)
-    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--steps", type=int, default=100)
+    p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", choices=["q_proj", "small"], default="q_proj")
+    p.add_argument("--tokens", type=int, default=0,
+                   help="calibration tokens (default: the workload's); a smaller "
+                        "full-path configuration for profiling captures")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
@@ -236,6 +239,8 @@ def run_ours(args, rank, world, local_rank):
     G.load_library()
     dev = torch.device("cuda", local_rank)
     spec = workload_spec(args.workload, rank)
+    if args.tokens:
+        spec = spec.with_(n_tokens=args.tokens, name=f"{spec.name}_n{args.tokens}")
     d, n, dr = spec.d_col, spec.n_tokens, spec.d_row
     cfg = G.make_config(bits=spec.bits, group_size=spec.group, sym=spec.sym,
                         block=spec.block, damp_rel=spec.damp)
@@ -350,10 +355,10 @@ def run_ours(args, rank, world, local_rank):
     }
     cpu = None
     if not args.no_cpu_baseline and world == 1:
-        res = oracle_sample(spec, x_host, w_host)
+        res = oracle_sample(spec, x_host, w_host, tokens=min(8192, n))
         cpu = {"value": dr * d / res["seconds_per_layer"], "unit": UNIT, "cores": cpu_cores(),
                "kind": "oracle", "sample": res["sample"],
-               "stage_s": {"hessian_full_est": res["hessian_s"] * n / 8192,
+               "stage_s": {"hessian_full_est": res["hessian_s"] * n / min(8192, n),
                            "factor": res["factor_s"], "quant_full_est": res["quant_s"] * dr / 32}}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,

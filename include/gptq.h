@@ -87,7 +87,8 @@ size_t gptq_workspace_size(int64_t d_row, int64_t d_col, const gptq_config* cfg)
  *         elements (ldx >= d, ldx % 8 == 0, X 16-byte aligned).  This is
  *         X^T of the page's d x n matrix, the layout a model's activations
  *         have.  Chunks of any size may be accumulated by repeated calls.
- *  d      % 8 == 0, 8 <= d <= 65536.   n >= 0 (n == 0 is a no-op).
+ *  d      % 8 == 0, 8 <= d <= 65536.   n >= 0 (n == 0 is a no-op and X may
+ *         then be NULL).
  * Summation order over tokens within one call is not fixed (split over
  * tokens with fp32 atomic adds), so results may differ in the last bits
  * between runs.  Asynchronous. */

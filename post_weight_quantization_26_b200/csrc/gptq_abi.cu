@@ -224,13 +224,13 @@ gptq_status gptq_device_status(void* stream) {
 
 gptq_status gptq_hessian_accumulate(float* H, const void* X, int64_t n, int64_t d, int64_t ldx,
                                     float scale, void* stream) {
-  if (!H || !X) return GPTQ_ERR_INVALID;
+  if (!H) return GPTQ_ERR_INVALID;
   if (d < 8 || d > 65536 || d % 8 != 0) return GPTQ_ERR_INVALID;
   if (n < 0 || n > (int64_t(1) << 31) - 1) return GPTQ_ERR_INVALID;
   if (ldx < d || ldx % 8 != 0) return GPTQ_ERR_INVALID;
-  if (!aligned(X, 16) || !aligned(H, 16)) return GPTQ_ERR_INVALID;
-  if (!std::isfinite(scale)) return GPTQ_ERR_INVALID;
-  if (n == 0) return GPTQ_OK;
+  if (!std::isfinite(scale) || !aligned(H, 16)) return GPTQ_ERR_INVALID;
+  if (n == 0) return GPTQ_OK;  // X may be NULL for an empty chunk
+  if (!X || !aligned(X, 16)) return GPTQ_ERR_INVALID;
   int num_sms = 0;
   gptq_status st = device_setup(&num_sms);
   if (st != GPTQ_OK) return st;

@@ -81,6 +81,7 @@ def test_hessian_accumulate_validation(lib):
     f = lib.gptq_hessian_accumulate
     assert f(None, FAKE, 16, 64, 64, 2.0, None) == 1
     assert f(FAKE, None, 16, 64, 64, 2.0, None) == 1
+    assert f(FAKE, None, 0, 64, 64, 2.0, None) == 0    # empty chunk, no data
     assert f(FAKE, FAKE, 16, 60, 64, 2.0, None) == 1   # d % 8
     assert f(FAKE, FAKE, 16, 64, 60, 2.0, None) == 1   # ldx < d
     assert f(FAKE, FAKE, 16, 64, 68, 2.0, None) == 1   # ldx % 8

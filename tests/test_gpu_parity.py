@@ -172,7 +172,7 @@ def _run_quantize(G, w, u32, bits, group, sym, block, dead=None):
     d_row, d_col = w.shape
     cfg = G.make_config(bits=bits, group_size=group, sym=sym, block=block)
     wt = torch.from_numpy(w.astype(np.float32)).cuda()
-    gt = torch.from_numpy(u32).cuda()
+    gt = torch.from_numpy(np.ascontiguousarray(u32, dtype=np.float32)).cuda()
     dm = None if dead is None else torch.from_numpy(dead.astype(np.uint8)).cuda()
     qw, sc, ze = G.alloc_outputs(d_row, d_col, cfg)
     ws = G.alloc_workspace(d_row, d_col, cfg)
