@@ -157,6 +157,37 @@ gptq_status gptq_dequant_check(const uint32_t* qweight, const float* scales,
                                double* loss, void* ws, size_t ws_bytes,
                                void* stream);
 
+/* Largest number of 128x128 tiles, ceil(d_row/128) * ceil(d_col/128), that
+ * gptq_dequant_check_noalloc accepts (e.g. 16384 x 65536 or 65536 x 16384). */
+#define GPTQ_NOALLOC_MAX_TILES 65536
+
+/* gptq_dequant_check without a workspace argument, for callers that cannot
+ * allocate device memory: for example a process whose device memory is all
+ * reserved up front by its own pool, or a code path where the device-wide
+ * synchronization of cudaMalloc is not allowed, and that has no workspace to
+ * pass.  The paper has no counterpart; this is an interface variant, not part
+ * of the method.
+ *  Same arguments, outputs and synchronization as gptq_dequant_check, minus
+ *  ws / ws_bytes.  Its scratch (one fp64 partial sum per 128x128 tile plus the
+ *  loss) lives in a fixed array of (GPTQ_NOALLOC_MAX_TILES + 32) doubles,
+ *  512 KB, in the library's device image: every GPU that loads the library
+ *  holds it until the process exits.  The call itself allocates nothing (no
+ *  cudaMalloc, cudaFree or allocating library routine).
+ *  Layers with more tiles than GPTQ_NOALLOC_MAX_TILES are rejected with
+ *  GPTQ_ERR_INVALID (and a message on stderr) before anything is launched.
+ *  The first call on a device looks up that array's device address (once per
+ *  device, with that device current); make that first call before any
+ *  stream capture.
+ *  All calls share the one array, which keeps the last call's contents; each
+ *  call overwrites every entry it later reads, so nothing needs clearing, but
+ *  calls that overlap on the GPU (other streams, other host threads) race on
+ *  it and must be serialized by the caller. */
+gptq_status gptq_dequant_check_noalloc(const uint32_t* qweight, const float* scales,
+                                       const uint8_t* zeros, const float* W,
+                                       const float* H, int64_t d_row, int64_t d_col,
+                                       const gptq_config* cfg, float* W_hat,
+                                       double* loss, void* stream);
+
 /* Synchronize `stream`, then return and clear the device status word that
  * kernels set when a bounded internal wait runs out (GPTQ_ERR_TIMEOUT). */
 gptq_status gptq_device_status(void* stream);

@@ -529,3 +529,84 @@ gptq_status gptq_dequant_check(const uint32_t* qweight, const float* scales, con
 }
 
 }  // extern "C"
+
+// ----------------------------------------------------------------------------
+// Loss check without a caller workspace: its scratch is this fixed device
+// array.  Host code must not pass g_noalloc_scratch itself to a kernel (on
+// the host the name is only a stand-in); it uses the device address that
+// cudaGetSymbolAddress returns, looked up once per device.
+static __device__ __align__(256) double g_noalloc_scratch[GPTQ_NOALLOC_MAX_TILES + 32];
+
+namespace {
+std::mutex g_noalloc_mu;
+double* g_noalloc_ptr[64] = {};
+
+gptq_status noalloc_scratch(double** out) {
+  int dev = 0;
+  GPTQ_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return GPTQ_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p) {
+      std::fprintf(stderr, "gptq: cudaGetSymbolAddress(no-alloc scratch) failed: %s\n",
+                   cudaGetErrorString(e));
+      return GPTQ_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = static_cast<double*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return GPTQ_OK;
+}
+}  // namespace
+
+extern "C" gptq_status gptq_dequant_check_noalloc(const uint32_t* qweight, const float* scales,
+                                                  const uint8_t* zeros, const float* W,
+                                                  const float* H, int64_t d_row, int64_t d_col,
+                                                  const gptq_config* cfg, float* W_hat,
+                                                  double* loss, void* stream) {
+  if (!qweight || !scales || !zeros) return GPTQ_ERR_INVALID;
+  if (d_row < 1 || d_row > (int64_t(1) << 24) || d_col < 32 || d_col % 32 != 0 ||
+      d_col > 65536)
+    return GPTQ_ERR_INVALID;
+  if (!config_ok(cfg, d_col)) return GPTQ_ERR_INVALID;
+  if (loss && (!W || !H)) return GPTQ_ERR_INVALID;
+  const int64_t tiles = ((d_row + 127) / 128) * ((d_col + 127) / 128);
+  if (tiles > GPTQ_NOALLOC_MAX_TILES) {
+    std::fprintf(stderr,
+                 "gptq: gptq_dequant_check_noalloc: %lld x %lld needs %lld tiles, more than "
+                 "GPTQ_NOALLOC_MAX_TILES (%d)\n",
+                 static_cast<long long>(d_row), static_cast<long long>(d_col),
+                 static_cast<long long>(tiles), GPTQ_NOALLOC_MAX_TILES);
+    return GPTQ_ERR_INVALID;
+  }
+  gptq_status st = device_setup(nullptr);
+  if (st != GPTQ_OK) return st;
+  double* scratch = nullptr;
+  st = noalloc_scratch(&scratch);
+  if (st != GPTQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int dr = static_cast<int>(d_row), dc = static_cast<int>(d_col);
+  const int g = cfg->group_size;
+  const int n_groups = g ? dc / g : 1;
+  if (W_hat) {
+    quant::dequant_kernel<<<1184, 256, 0, s>>>(qweight, scales, zeros, dr, dc, cfg->bits, g,
+                                               n_groups, W_hat);
+    GPTQ_LAUNCH_CHECK();
+  }
+  if (loss) {
+    double* partials = scratch;                        // one slot per tile, all rewritten
+    double* dloss = scratch + GPTQ_NOALLOC_MAX_TILES;  // written by the final sum
+    const dim3 grid((dr + 127) / 128, (dc + 127) / 128);
+    quant::loss_tiles_kernel<<<grid, 256, 0, s>>>(qweight, scales, zeros, W, H, dr, dc,
+                                                  cfg->bits, g, n_groups, partials);
+    GPTQ_LAUNCH_CHECK();
+    quant::sum_partials_kernel<<<1, 1024, 0, s>>>(partials, static_cast<int>(grid.x * grid.y),
+                                                  dloss);
+    GPTQ_LAUNCH_CHECK();
+    GPTQ_CUDA_TRY(cudaMemcpyAsync(loss, dloss, 8, cudaMemcpyDeviceToHost, s));
+  }
+  GPTQ_CUDA_TRY(cudaStreamSynchronize(s));
+  return GPTQ_OK;
+}

@@ -24,7 +24,9 @@ STATUS_NAMES = {0: "GPTQ_OK", 1: "GPTQ_ERR_INVALID", 2: "GPTQ_ERR_NOT_SPD",
 
 EXPORTED = ("gptq_workspace_size", "gptq_hessian_accumulate",
             "gptq_prepare_hinv", "gptq_quantize_layer", "gptq_dequant_check",
-            "gptq_device_status", "gptq_status_string", "gptq_launch_count")
+            "gptq_device_status", "gptq_status_string", "gptq_launch_count",
+            "gptq_dequant_check_noalloc")
+NOALLOC_MAX_TILES = 65536  # GPTQ_NOALLOC_MAX_TILES in include/gptq.h
 
 
 class GptqError(RuntimeError):
@@ -73,6 +75,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gptq_dequant_check.argtypes = [P, P, P, P, P, I64, I64, cfgp, P,
                                        ctypes.POINTER(D), P, SZ, P]
     lib.gptq_dequant_check.restype = I
+    lib.gptq_dequant_check_noalloc.argtypes = [P, P, P, P, P, I64, I64, cfgp, P,
+                                               ctypes.POINTER(D), P]
+    lib.gptq_dequant_check_noalloc.restype = I
     lib.gptq_device_status.argtypes = [P]
     lib.gptq_device_status.restype = I
     lib.gptq_launch_count.argtypes = []
@@ -167,6 +172,22 @@ def gptq_dequant_check(qweight, scales, zeros, W, H, cfg: GptqConfig,
         ctypes.byref(loss) if want_loss else None, _ptr(ws),
         0 if ws is None else ws.numel(), _stream(stream))
     _check(st, "gptq_dequant_check")
+    return loss.value if want_loss else None
+
+
+def gptq_dequant_check_noalloc(qweight, scales, zeros, W, H, cfg: GptqConfig,
+                               W_hat=None, want_loss: bool = True, stream=None):
+    """gptq_dequant_check for callers that cannot allocate device memory:
+    no workspace argument; the library's fixed 512 KB device array serves as
+    scratch (see include/gptq.h for the size limit and the rules on
+    overlapping calls).  Returns the layer loss (or None)."""
+    d_row, d_col = W.shape if W is not None else W_hat.shape
+    loss = ctypes.c_double(float("nan"))
+    st = load_library().gptq_dequant_check_noalloc(
+        _ptr(qweight), _ptr(scales), _ptr(zeros), _ptr(W), _ptr(H), d_row,
+        d_col, ctypes.byref(cfg), _ptr(W_hat),
+        ctypes.byref(loss) if want_loss else None, _stream(stream))
+    _check(st, "gptq_dequant_check_noalloc")
     return loss.value if want_loss else None
 
 
