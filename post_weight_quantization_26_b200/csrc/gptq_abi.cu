@@ -54,14 +54,28 @@ std::atomic<uint64_t> g_launches{0};
   } while (0)
 
 // ------------------------------------------------------------ device setup
+constexpr int kEvents = 10;  // fork, join, 4 block-step and 4 trailing-update events
+
 struct DeviceInfo {
   bool ready = false;
   int num_sms = 0;
+  // The column sweep runs the block steps on the caller's stream and the
+  // trailing updates on this auxiliary stream, joined by events; qmu keeps
+  // calls from several host threads from interleaving on them.
+  cudaStream_t aux = nullptr;
+  cudaEvent_t ev[kEvents] = {};
+  std::mutex qmu;
 };
 
 std::mutex g_mu;
 DeviceInfo g_dev[64];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+DeviceInfo* current_device_info() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  return &g_dev[dev];
+}
 
 gptq_status device_setup(int* num_sms) {
   int dev = 0;
@@ -74,27 +88,30 @@ gptq_status device_setup(int* num_sms) {
     GPTQ_CUDA_TRY(cudaFuncSetAttribute(syrk::syrk_bf16_tcgen05_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        syrk::SMEM_BYTES));
-    GPTQ_CUDA_TRY(cudaFuncSetAttribute(chol::dgemm_grouped_kernel,
+    GPTQ_CUDA_TRY(cudaFuncSetAttribute(chol::dgemm_nt_kernel<128, 2>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       chol::GEMM_SMEM));
-    GPTQ_CUDA_TRY(cudaFuncSetAttribute(chol::leaf_potrf_inv_kernel,
+                                       chol::gemm_smem<128>()));
+    GPTQ_CUDA_TRY(cudaFuncSetAttribute(chol::dgemm_nt_kernel<64, 2>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       chol::gemm_smem<64>()));
+    GPTQ_CUDA_TRY(cudaFuncSetAttribute(chol::dgemm_nt_kernel<32, 1>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       chol::gemm_smem<32>()));
+    GPTQ_CUDA_TRY(cudaFuncSetAttribute(chol::leaf_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        chol::LEAF_SMEM));
-    GPTQ_CUDA_TRY(cudaFuncSetAttribute(quant::block_quant_kernel<128, 0>,
+    GPTQ_CUDA_TRY(cudaFuncSetAttribute(quant::block_step_kernel<128>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       quant::block_quant_smem<128>()));
-    GPTQ_CUDA_TRY(cudaFuncSetAttribute(quant::block_quant_kernel<128, 32>,
+                                       quant::block_step_smem<128>()));
+    GPTQ_CUDA_TRY(cudaFuncSetAttribute(quant::block_step_kernel<64>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       quant::block_quant_smem<128>()));
-    GPTQ_CUDA_TRY(cudaFuncSetAttribute(quant::block_quant_kernel<128, 64>,
+                                       quant::block_step_smem<64>()));
+    GPTQ_CUDA_TRY(cudaFuncSetAttribute(quant::block_step_kernel<32>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       quant::block_quant_smem<128>()));
-    GPTQ_CUDA_TRY(cudaFuncSetAttribute(quant::block_quant_kernel<64, 0>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       quant::block_quant_smem<64>()));
-    GPTQ_CUDA_TRY(cudaFuncSetAttribute(quant::block_quant_kernel<64, 32>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       quant::block_quant_smem<64>()));
+                                       quant::block_step_smem<32>()));
+    GPTQ_CUDA_TRY(cudaStreamCreateWithFlags(&di.aux, cudaStreamNonBlocking));
+    for (int i = 0; i < kEvents; ++i)
+      GPTQ_CUDA_TRY(cudaEventCreateWithFlags(&di.ev[i], cudaEventDisableTiming));
     if (!g_encode) {
       cudaDriverEntryPointQueryResult q;
       void* fn = nullptr;
@@ -126,7 +143,7 @@ bool config_ok(const gptq_config* c, int64_t d_col) {
 
 // ---------------------------------------------------------- workspace map
 struct PrepareWs {
-  size_t stats, istat, pivot, A, Xd, total;
+  size_t stats, istat, pivot, A, Mt, Xd, total;
 };
 PrepareWs prepare_layout(int64_t d) {
   PrepareWs w{};
@@ -135,6 +152,7 @@ PrepareWs prepare_layout(int64_t d) {
   w.istat = off; off = align_up(off + 8);
   w.pivot = off; off = align_up(off + 8);
   w.A = off; off = align_up(off + static_cast<size_t>(d) * d * 8);
+  w.Mt = off; off = align_up(off + static_cast<size_t>(d) * d * 8);
   const int64_t nt = (d + chol::NB - 1) / chol::NB;
   w.Xd = off; off = align_up(off + static_cast<size_t>(nt) * chol::NB * chol::NB * 8);
   w.total = off;
@@ -142,13 +160,14 @@ PrepareWs prepare_layout(int64_t d) {
 }
 
 struct QuantWs {
-  size_t Wk, E, total;
+  size_t Wk, E0, E1, total;
 };
 QuantWs quant_layout(int64_t d_row, int64_t d_col, int block) {
   QuantWs w{};
   size_t off = 0;
   w.Wk = off; off = align_up(off + static_cast<size_t>(d_row) * d_col * 4);
-  w.E = off; off = align_up(off + static_cast<size_t>(d_row) * block * 4);
+  w.E0 = off; off = align_up(off + static_cast<size_t>(d_row) * block * 4);
+  w.E1 = off; off = align_up(off + static_cast<size_t>(d_row) * block * 4);
   w.total = off;
   return w;
 }
@@ -184,6 +203,39 @@ void choose_split(int ntiles, int n, int num_sms, int* split_tokens, int* nsplit
   const int kb_per = (nkb + best_s - 1) / best_s;
   *split_tokens = kb_per * syrk::BK;
   *nsplit = (nkb + kb_per - 1) / kb_per;
+}
+
+}  // namespace
+
+namespace {
+
+// Launch the grouped NT DGEMM with TM-row tiles: persistent CTAs, at most
+// one per SM.  Problems with an empty output are dropped.
+template <int TM, int WGM>
+gptq_status launch_nt(const std::vector<chol::GemmProblem>& probs, cudaStream_t s) {
+  int num_sms = 148;
+  gptq_status st = device_setup(&num_sms);
+  if (st != GPTQ_OK) return st;
+  size_t i = 0;
+  while (i < probs.size()) {
+    chol::GemmBatch b{};
+    int tiles = 0;
+    while (i < probs.size() && b.count < chol::MAXP) {
+      const chol::GemmProblem& q = probs[i++];
+      if (q.M <= 0 || q.N <= 0) continue;
+      const int tm = (q.M + TM - 1) / TM, tn = (q.N + chol::TN - 1) / chol::TN;
+      b.tile_start[b.count] = tiles;
+      b.p[b.count++] = q;
+      tiles += q.lower_only ? tm * (tm + 1) / 2 : tm * tn;
+    }
+    b.tile_start[b.count] = tiles;
+    const int grid = std::min(tiles, num_sms);
+    if (grid > 0) {
+      chol::dgemm_nt_kernel<TM, WGM><<<grid, chol::GEMM_THREADS, chol::gemm_smem<TM>(), s>>>(b);
+      GPTQ_LAUNCH_CHECK();
+    }
+  }
+  return GPTQ_OK;
 }
 
 }  // namespace
@@ -269,51 +321,6 @@ gptq_status gptq_hessian_accumulate(float* H, const void* X, int64_t n, int64_t 
   return GPTQ_OK;
 }
 
-namespace {
-
-gptq_status launch_gemm_batch(std::vector<chol::GemmProblem>& probs, cudaStream_t s) {
-  size_t i = 0;
-  while (i < probs.size()) {
-    chol::GemmBatch b{};
-    int tiles = 0;
-    b.count = 0;
-    while (i < probs.size() && b.count < chol::MAXP) {
-      const chol::GemmProblem& q = probs[i];
-      const int tm = (q.M + chol::TM - 1) / chol::TM, tn = (q.N + chol::TN - 1) / chol::TN;
-      const int nt = q.lower_only ? tm * (tm + 1) / 2 : tm * tn;
-      if (q.M > 0 && q.N > 0) {
-        b.tile_start[b.count] = tiles;
-        b.p[b.count] = q;
-        tiles += nt;
-        ++b.count;
-      }
-      ++i;
-    }
-    b.tile_start[b.count] = tiles;
-    if (tiles > 0) {
-      chol::dgemm_grouped_kernel<<<tiles, chol::GEMM_THREADS, chol::GEMM_SMEM, s>>>(b);
-      GPTQ_LAUNCH_CHECK();
-    }
-  }
-  return GPTQ_OK;
-}
-
-struct Node {
-  int a, m, b, height;
-};
-
-int build_tree(int a, int b, std::vector<Node>& out) {
-  // nodes over [a, b) in units of NB blocks (a, b are block indices)
-  if (b - a <= 1) return 0;
-  const int m = a + (b - a + 1) / 2;
-  const int hl = build_tree(a, m, out);
-  const int hr = build_tree(m, b, out);
-  const int h = 1 + std::max(hl, hr);
-  out.push_back(Node{a, m, b, h});
-  return h;
-}
-
-}  // namespace
 
 gptq_status gptq_prepare_hinv(const float* H, int64_t d, double damp_rel, float* G,
                               uint8_t* dead_mask, void* ws, size_t ws_bytes,
@@ -332,9 +339,12 @@ gptq_status gptq_prepare_hinv(const float* H, int64_t d, double damp_rel, float*
   int* istat = reinterpret_cast<int*>(base + L.istat);
   long long* pivot = reinterpret_cast<long long*>(base + L.pivot);
   double* A = reinterpret_cast<double*>(base + L.A);
+  double* Mt = reinterpret_cast<double*>(base + L.Mt);
   double* Xd = reinterpret_cast<double*>(base + L.Xd);
   const int di = static_cast<int>(d);
-  const int nt = (di + chol::NB - 1) / chol::NB;
+  const int NB = chol::NB;
+  const int nt = (di + NB - 1) / NB;
+  auto at = [&](double* m, int r, int c) { return m + static_cast<size_t>(r) * di + c; };
 
   GPTQ_CUDA_TRY(cudaMemsetAsync(pivot, 0xFF, 8, s));
   chol::diag_stats_kernel<<<1, 1024, 0, s>>>(H, di, damp_rel, dead_mask, stats, istat);
@@ -344,80 +354,94 @@ gptq_status gptq_prepare_hinv(const float* H, int64_t d, double damp_rel, float*
     chol::reverse_damp_fill_kernel<<<grid, 256, 0, s>>>(H, di, stats, A);
     GPTQ_LAUNCH_CHECK();
   }
-  // blocked right-looking Cholesky of A (the reversed, damped H)
-  for (int k = 0; k < nt; ++k) {
-    const int k0 = k * chol::NB;
-    const int nk = std::min(chol::NB, di - k0);
-    double* Xk = Xd + static_cast<size_t>(k) * chol::NB * chol::NB;
-    chol::leaf_potrf_inv_kernel<<<1, chol::LEAF_THREADS, chol::LEAF_SMEM, s>>>(A, di, k0, nk, Xk,
-                                                                                 pivot);
-    GPTQ_LAUNCH_CHECK();
-    const int rest = di - k0 - nk;
-    if (rest <= 0) continue;
-    std::vector<chol::GemmProblem> v(1);
-    chol::GemmProblem& pn = v[0];
-    pn = chol::GemmProblem{};
-    pn.A = A + static_cast<size_t>(k0 + nk) * di + k0;
-    pn.lda = di;
-    pn.a_trans = 0;
-    pn.B = Xk;
-    pn.ldb = chol::NB;
-    pn.b_trans = 1;
-    pn.C = A + static_cast<size_t>(k0 + nk) * di + k0;
-    pn.ldc = di;
-    pn.M = rest; pn.N = nk; pn.K = nk;
-    pn.alpha = 1.0; pn.beta = 0.0;
-    st = launch_gemm_batch(v, s);
-    if (st != GPTQ_OK) return st;
-    chol::GemmProblem up{};
-    up.A = A + static_cast<size_t>(k0 + nk) * di + k0;
-    up.lda = di;
-    up.a_trans = 0;
-    up.B = A + static_cast<size_t>(k0 + nk) * di + k0;
-    up.ldb = di;
-    up.b_trans = 1;
-    up.C = A + static_cast<size_t>(k0 + nk) * di + (k0 + nk);
-    up.ldc = di;
-    up.M = rest; up.N = rest; up.K = nk;
-    up.lower_only = 1;
-    up.alpha = -1.0; up.beta = 1.0;
-    v[0] = up;
-    st = launch_gemm_batch(v, s);
-    if (st != GPTQ_OK) return st;
-  }
-  // triangular inverse: diagonal blocks from the leaves, then by tree height
-  chol::place_diag_inverses_kernel<<<nt, 256, 0, s>>>(A, di, Xd);
+  DeviceInfo* dinfo = current_device_info();
+  if (!dinfo) return GPTQ_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(dinfo->qmu);
+  cudaStream_t aux = dinfo->aux;
+  cudaEvent_t evP[2] = {dinfo->ev[2], dinfo->ev[3]};
+  cudaEvent_t evL[2] = {dinfo->ev[4], dinfo->ev[5]};
+  auto leaf = [&](int off, int n, cudaStream_t st) {
+    chol::leaf_kernel<<<1, chol::LEAF_THREADS, chol::LEAF_SMEM, st>>>(
+        A, Mt, Xd + static_cast<size_t>(off / NB) * NB * NB, di, off, n, pivot);
+  };
+  leaf(0, std::min(NB, di), s);
   GPTQ_LAUNCH_CHECK();
-  std::vector<Node> nodes;
-  const int height = build_tree(0, nt, nodes);
-  for (int h = 1; h <= height; ++h) {
-    std::vector<chol::GemmProblem> g1, g2;
-    for (const Node& nd : nodes) {
-      if (nd.height != h) continue;
-      const int a = nd.a * chol::NB, m = nd.m * chol::NB, b = std::min(nd.b * chol::NB, di);
-      chol::GemmProblem p1{};  // T^T = X11^T L21^T stored at A[a:m, m:b]
-      p1.A = A + static_cast<size_t>(a) * di + a; p1.lda = di; p1.a_trans = 1; p1.kmode = 2;
-      p1.B = A + static_cast<size_t>(m) * di + a; p1.ldb = di; p1.b_trans = 1;
-      p1.C = A + static_cast<size_t>(a) * di + m; p1.ldc = di;
-      p1.M = m - a; p1.N = b - m; p1.K = m - a;
-      p1.alpha = 1.0; p1.beta = 0.0;
-      g1.push_back(p1);
-      chol::GemmProblem p2{};  // X21 = -X22 T
-      p2.A = A + static_cast<size_t>(m) * di + m; p2.lda = di; p2.a_trans = 0; p2.kmode = 1;
-      p2.B = A + static_cast<size_t>(a) * di + m; p2.ldb = di; p2.b_trans = 1;
-      p2.C = A + static_cast<size_t>(m) * di + a; p2.ldc = di;
-      p2.M = b - m; p2.N = m - a; p2.K = b - m;
-      p2.alpha = -1.0; p2.beta = 0.0;
-      g2.push_back(p2);
+  // Step k: P_k (caller's stream) forms the panel and rescales M's row
+  // block k; then the auxiliary stream updates the next diagonal block (D_k)
+  // and factors it (leaf k+1) while the caller's stream runs the rest of the
+  // trailing update U_k; P_{k+1} waits for both.
+  for (int k = 0; k < nt; ++k) {
+    const int k0 = k * NB, nk = std::min(NB, di - k0), k1 = k0 + nk, rest = di - k1;
+    double* Xk = Xd + static_cast<size_t>(k) * NB * NB;
+    std::vector<chol::GemmProblem> pk;
+    if (rest > 0) {
+      chol::GemmProblem q{};  // L21 = A21 X_kk^T
+      q.A = at(A, k1, k0); q.lda = di; q.B = Xk; q.ldb = NB; q.C = at(A, k1, k0); q.ldc = di;
+      q.M = rest; q.N = nk; q.K = nk; q.alpha = 1.0; q.beta = 0.0;
+      pk.push_back(q);
     }
-    st = launch_gemm_batch(g1, s);
+    if (k0 > 0) {
+      chol::GemmProblem q{};  // Mt[:k0, block k] <- Mt[:k0, block k] X_kk^T
+      q.A = at(Mt, 0, k0); q.lda = di; q.B = Xk; q.ldb = NB; q.C = at(Mt, 0, k0); q.ldc = di;
+      q.M = k0; q.N = nk; q.K = nk; q.alpha = 1.0; q.beta = 0.0;
+      pk.push_back(q);
+    }
+    const int prow = rest + k0;
+    if (prow >= 148 * 128) st = launch_nt<128, 2>(pk, s);
+    else if (prow >= 148 * 64) st = launch_nt<64, 2>(pk, s);
+    else st = launch_nt<32, 1>(pk, s);
     if (st != GPTQ_OK) return st;
-    st = launch_gemm_batch(g2, s);
+    if (rest <= 0) break;
+    const int n1 = std::min(NB, rest);  // next diagonal block
+    GPTQ_CUDA_TRY(cudaEventRecord(evP[k & 1], s));
+    GPTQ_CUDA_TRY(cudaStreamWaitEvent(aux, evP[k & 1], 0));
+    {
+      std::vector<chol::GemmProblem> dk(1);
+      chol::GemmProblem& q = dk[0];  // D_k: A_{k+1,k+1} -= L_{k+1} L_{k+1}^T
+      q = chol::GemmProblem{};
+      q.A = at(A, k1, k0); q.lda = di; q.B = at(A, k1, k0); q.ldb = di;
+      q.C = at(A, k1, k1); q.ldc = di;
+      q.M = n1; q.N = n1; q.K = nk; q.alpha = -1.0; q.beta = 1.0;
+      st = launch_nt<32, 1>(dk, aux);
+      if (st != GPTQ_OK) return st;
+      leaf(k1, n1, aux);
+      GPTQ_LAUNCH_CHECK();
+      GPTQ_CUDA_TRY(cudaEventRecord(evL[k & 1], aux));
+    }
+    std::vector<chol::GemmProblem> uk;
+    if (rest > n1) {
+      chol::GemmProblem q{};  // rows below the next diagonal block, its columns
+      q.A = at(A, k1 + n1, k0); q.lda = di; q.B = at(A, k1, k0); q.ldb = di;
+      q.C = at(A, k1 + n1, k1); q.ldc = di;
+      q.M = rest - n1; q.N = n1; q.K = nk; q.alpha = -1.0; q.beta = 1.0;
+      uk.push_back(q);
+      chol::GemmProblem r{};  // the rest of the trailing matrix, lower tiles
+      r.A = at(A, k1 + n1, k0); r.lda = di; r.B = at(A, k1 + n1, k0); r.ldb = di;
+      r.C = at(A, k1 + n1, k1 + n1); r.ldc = di;
+      r.M = rest - n1; r.N = rest - n1; r.K = nk; r.lower_only = 1; r.alpha = -1.0; r.beta = 1.0;
+      uk.push_back(r);
+    }
+    if (k0 > 0) {
+      chol::GemmProblem q{};  // Mt[:k0, k1:] -= Mt[:k0, block k] L21^T
+      q.A = at(Mt, 0, k0); q.lda = di; q.B = at(A, k1, k0); q.ldb = di;
+      q.C = at(Mt, 0, k1); q.ldc = di;
+      q.M = k0; q.N = rest; q.K = nk; q.alpha = -1.0; q.beta = 1.0;
+      uk.push_back(q);
+    }
+    {
+      chol::GemmProblem q{};  // Mt[block k, k1:] = -X_kk^T L21^T (first write)
+      q.A = at(Mt, k0, k0); q.lda = di; q.B = at(A, k1, k0); q.ldb = di;
+      q.C = at(Mt, k0, k1); q.ldc = di;
+      q.M = nk; q.N = rest; q.K = nk; q.alpha = -1.0; q.beta = 0.0;
+      uk.push_back(q);
+    }
+    st = launch_nt<128, 2>(uk, s);
     if (st != GPTQ_OK) return st;
+    GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, evL[k & 1], 0));  // X_{k+1} for P_{k+1}
   }
   {
-    dim3 grid((di + 255) / 256, di);
-    chol::write_g_kernel<<<grid, 256, 0, s>>>(A, di, G);
+    dim3 grid((di + 31) / 32, (di + 31) / 32);
+    chol::write_g_kernel<<<grid, dim3(32, 8), 0, s>>>(Mt, di, G);
     GPTQ_LAUNCH_CHECK();
   }
   long long host_pivot = -1;
@@ -450,41 +474,63 @@ gptq_status gptq_quantize_layer(const float* W, int64_t d_row, int64_t d_col, co
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* base = static_cast<uint8_t*>(ws);
   float* Wk = reinterpret_cast<float*>(base + L.Wk);
-  float* E = reinterpret_cast<float*>(base + L.E);
+  float* Ebuf[2] = {reinterpret_cast<float*>(base + L.E0), reinterpret_cast<float*>(base + L.E1)};
   const int dr = static_cast<int>(d_row), dc = static_cast<int>(d_col);
   const int B = cfg->block, g = cfg->group_size;
   const int n_groups = g ? dc / g : 1;
   const int per_channel = g == 0;
+  DeviceInfo* di = current_device_info();
+  if (!di) return GPTQ_ERR_CUDA;
 
   quant::prepare_rows_kernel<<<(dr + 7) / 8, 256, 0, s>>>(W, Wk, dead_mask, dr, dc, cfg->bits,
                                                            cfg->sym, per_channel, scales, zeros);
   GPTQ_LAUNCH_CHECK();
-  const int gs_inblock = (g > 0 && g < B) ? g : 0;
+  // Block j: the step kernel Q_j (caller's stream) applies E_{j-1} to block j
+  // and quantizes it; the trailing kernel T_j (auxiliary stream) applies E_j
+  // to the columns right of block j+1.  Q_j needs T_{j-2} (it finished
+  // block j's earlier updates; also frees E buffer j%2); T_j needs Q_j.  So
+  // Q_{j+1} overlaps T_j.
+  std::lock_guard<std::mutex> lk(di->qmu);
+  cudaEvent_t ev_fork = di->ev[0], ev_join = di->ev[1];
+  cudaEvent_t* evQ = di->ev + 2;
+  cudaEvent_t* evT = di->ev + 6;
+  GPTQ_CUDA_TRY(cudaEventRecord(ev_fork, s));
+  GPTQ_CUDA_TRY(cudaStreamWaitEvent(di->aux, ev_fork, 0));
+  const int nblk = (dc + B - 1) / B;
   const dim3 qgrid((dr + quant::QROWS - 1) / quant::QROWS);
-  for (int j0 = 0; j0 < dc; j0 += B) {
-    const int ncols = std::min(B, dc - j0);
-#define GPTQ_BQ(BB, GSV)                                                                     \
-  quant::block_quant_kernel<BB, GSV><<<qgrid, quant::QTHREADS, quant::block_quant_smem<BB>(), s>>>( \
-      Wk, dr, dc, j0, ncols, G, E, qweight, scales, zeros, cfg->bits, cfg->sym, g, n_groups,   \
-      per_channel)
-    if (B == 128 && gs_inblock == 0) GPTQ_BQ(128, 0);
-    else if (B == 128 && gs_inblock == 32) GPTQ_BQ(128, 32);
-    else if (B == 128 && gs_inblock == 64) GPTQ_BQ(128, 64);
-    else if (B == 64 && gs_inblock == 0) GPTQ_BQ(64, 0);
-    else if (B == 64 && gs_inblock == 32) GPTQ_BQ(64, 32);
-    else if (B == 32) GPTQ_BQ(32, 0);
-    else return GPTQ_ERR_INVALID;
-#undef GPTQ_BQ
+  std::vector<char> t_done(nblk, 0);
+  for (int jb = 0; jb < nblk; ++jb) {
+    const int j0 = jb * B, ncols = std::min(B, dc - j0);
+    if (jb >= 2 && t_done[jb - 2]) GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, evT[(jb - 2) % 4], 0));
+    if (g > B && j0 % g == 0 && jb >= 1 && t_done[jb - 1])  // group params read columns ahead
+      GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, evT[(jb - 1) % 4], 0));
+    const float* Ep = jb > 0 ? Ebuf[(jb - 1) & 1] : nullptr;
+    const int jp0 = jb > 0 ? j0 - B : -1;
+    float* Ec = Ebuf[jb & 1];
+#define GPTQ_STEP(BB)                                                                        \
+  quant::block_step_kernel<BB><<<qgrid, quant::QTHREADS, quant::block_step_smem<BB>(), s>>>( \
+      Wk, dr, dc, j0, ncols, G, Ep, jp0, Ec, qweight, scales, zeros, cfg->bits, cfg->sym, g,    \
+      n_groups, per_channel)
+    if (B == 128) GPTQ_STEP(128);
+    else if (B == 64) GPTQ_STEP(64);
+    else GPTQ_STEP(32);
+#undef GPTQ_STEP
     GPTQ_LAUNCH_CHECK();
-    const int j1 = j0 + ncols;
-    if (j1 < dc) {
-      const int N = dc - j1;
+    GPTQ_CUDA_TRY(cudaEventRecord(evQ[jb % 4], s));
+    const int n0 = j0 + 2 * B;  // block jb+1 is updated by Q_{jb+1} itself
+    if (n0 < dc) {
+      const int N = dc - n0;
+      GPTQ_CUDA_TRY(cudaStreamWaitEvent(di->aux, evQ[jb % 4], 0));
       const dim3 ugrid((dr + quant::UT - 1) / quant::UT, (N + quant::UT - 1) / quant::UT);
-      quant::trailing_update_kernel<<<ugrid, quant::UTHREADS, 0, s>>>(
-          Wk + j1, E, G + static_cast<size_t>(j0) * dc + j1, dr, N, B, dc, dc);
+      quant::trailing_update_kernel<<<ugrid, quant::UTHREADS, 0, di->aux>>>(
+          Wk + n0, Ec, G + static_cast<size_t>(j0) * dc + n0, dr, N, ncols, dc, dc);
       GPTQ_LAUNCH_CHECK();
+      GPTQ_CUDA_TRY(cudaEventRecord(evT[jb % 4], di->aux));
+      t_done[jb] = 1;
     }
   }
+  GPTQ_CUDA_TRY(cudaEventRecord(ev_join, di->aux));
+  GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, ev_join, 0));
   return GPTQ_OK;
 }
 

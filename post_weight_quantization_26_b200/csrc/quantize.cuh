@@ -83,159 +83,237 @@ __global__ void prepare_rows_kernel(const float* __restrict__ W, float* __restri
   }
 }
 
+// ------------------------------------------------------------- block step
+// One block of B columns for a slab of QROWS rows (4 threads per row; thread
+// t of a row owns columns 16c + 4t .. 16c + 4t + 3 of the block):
+//   (a) if a previous block exists, apply its errors to this block only:
+//       W[rows, blk] -= E_prev[rows] * G[prev blk, blk]  (the columns
+//       further right get them from the trailing-update kernel);
+//   (b) quantize the block column by column in 16-column sub-blocks: per
+//       column the owner codes w_q, e = (w_q - w^_q) / G_qq is broadcast to
+//       the row's 4 threads, each updates its later columns of the
+//       sub-block in registers; after each sub-block one rank-16 update
+//       carries its errors to the rest of the block (same sums as
+//       column-at-a-time, grouped);
+//   (c) bit-pack the block's codes and write E for the trailing update.
+// Group parameters are taken from the current weights when a group's first
+// column is reached (always a sub-block start, as groups are multiples of 32).
 constexpr int QROWS = 32;            // rows per CTA
 constexpr int QTHREADS = QROWS * 4;  // 4 threads per row
 
 template <int B>
-constexpr int block_quant_smem() {
-  return B * B * 4 + B * 4 + QROWS * B;
+struct StepSmem {
+  static constexpr int LDG = B + 4;  // padded rows (floats)
+  static constexpr int G_OFF = 0;
+  static constexpr int W_OFF = G_OFF + B * LDG * 4;
+  static constexpr int E_OFF = W_OFF + QROWS * LDG * 4;
+  static constexpr int INV_OFF = E_OFF + QROWS * LDG * 4;
+  static constexpr int C_OFF = INV_OFF + B * 4;
+  static constexpr int BYTES = C_OFF + QROWS * B;
+};
+
+template <int B>
+constexpr int block_step_smem() { return StepSmem<B>::BYTES; }
+
+template <int B>
+__device__ __forceinline__ void stage_rows(float* dst, const float* src, long long ld, int r0,
+                                           int d_row, int ncols, int tid) {
+  // QROWS x ncols floats -> dst (row stride LDG); rows beyond d_row are zero
+  constexpr int LDG = StepSmem<B>::LDG;
+  const int cpr = ncols / 4;
+  for (int c = tid; c < QROWS * cpr; c += QTHREADS) {
+    const int rr = c / cpr, k = (c - rr * cpr) * 4;
+    const bool ok = r0 + rr < d_row;
+    const float* sp = ok ? src + static_cast<long long>(r0 + rr) * ld + k : src;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst + rr * LDG + k)),
+                 "l"(sp), "r"(ok ? 16 : 0)
+                 : "memory");
+  }
 }
 
-// Mode flags for the group handling at the block start (GS == 0 variants):
-//   pc_mode 1: parameters per output channel, precomputed;
-//   pc_mode 0: group_size is a multiple of B: a group starts here when
-//              j0 % group == 0 (parameters over columns [j0, j0+group) of the
-//              current W, the part beyond this block read from memory),
-//              otherwise the group's parameters were written by an earlier block.
-template <int B, int GS>
+template <int B>
+__device__ __forceinline__ void stage_gblock(float* dst, const float* G, int d_col, int r0,
+                                             int c0, int nrows, int ncols, int tid) {
+  constexpr int LDG = StepSmem<B>::LDG;
+  const int cpr = ncols / 4;
+  for (int c = tid; c < nrows * cpr; c += QTHREADS) {
+    const int rr = c / cpr, k = (c - rr * cpr) * 4;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, 16;" ::"r"(smem_u32(dst + rr * LDG + k)),
+                 "l"(G + static_cast<long long>(r0 + rr) * d_col + c0 + k)
+                 : "memory");
+  }
+}
+
+template <int B>
 __global__ void __launch_bounds__(QTHREADS)
-block_quant_kernel(const float* __restrict__ Wk, int d_row, int d_col, int j0, int ncols,
-                   const float* __restrict__ G, float* __restrict__ E,
-                   uint32_t* __restrict__ qweight, float* __restrict__ scales,
-                   uint8_t* __restrict__ zeros, int bits, int sym, int group, int n_groups,
-                   int pc_mode) {
-  static_assert(B % 16 == 0 && (GS == 0 || (GS % 16 == 0 && B % GS == 0)), "shape");
-  constexpr int V = B / 4;       // values per thread
-  constexpr int NCH = B / 16;    // 16-column chunks; thread t owns columns 16c+4t..16c+4t+3
+block_step_kernel(const float* __restrict__ Wk, int d_row, int d_col, int j0, int ncols,
+                  const float* __restrict__ G, const float* __restrict__ Eprev, int jp0,
+                  float* __restrict__ Ecur, uint32_t* __restrict__ qweight,
+                  float* __restrict__ scales, uint8_t* __restrict__ zeros, int bits, int sym,
+                  int group, int n_groups, int pc_mode) {
+  using L = StepSmem<B>;
+  constexpr int LDG = L::LDG;
   extern __shared__ __align__(16) uint8_t qsm[];
-  float* gs = reinterpret_cast<float*>(qsm);  // B x B block of G
-  float* inv_diag = gs + B * B;
-  uint8_t* cstage = reinterpret_cast<uint8_t*>(inv_diag + B);  // QROWS x B codes
+  float* Gs = reinterpret_cast<float*>(qsm + L::G_OFF);
+  float* Ws = reinterpret_cast<float*>(qsm + L::W_OFF);
+  float* Es = reinterpret_cast<float*>(qsm + L::E_OFF);
+  float* invd = reinterpret_cast<float*>(qsm + L::INV_OFF);
+  uint8_t* codes = qsm + L::C_OFF;
 
   const int tid = threadIdx.x;
   const int rloc = tid >> 2, t = tid & 3;
-  const int lane = tid & 31;
-  const int qbase = lane & ~3;
-  const int r = blockIdx.x * QROWS + rloc;
+  const int lane = tid & 31, qbase = lane & ~3;
+  const int r0 = blockIdx.x * QROWS;
+  const int r = r0 + rloc;
   const bool rv = r < d_row;
 
-  for (int idx = tid; idx < B * B / 4; idx += QTHREADS) {
-    const int q = (idx * 4) / B, k = (idx * 4) % B;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (q < ncols && k < ncols)
-      v = *reinterpret_cast<const float4*>(G + static_cast<size_t>(j0 + q) * d_col + j0 + k);
-    reinterpret_cast<float4*>(gs)[idx] = v;
+  stage_rows<B>(Ws, Wk + j0, d_col, r0, d_row, ncols, tid);
+  if (jp0 >= 0) {
+    stage_rows<B>(Es, Eprev, B, r0, d_row, B, tid);
+    stage_gblock<B>(Gs, G, d_col, jp0, j0, B, ncols, tid);
+  } else {
+    stage_gblock<B>(Gs, G, d_col, j0, j0, ncols, ncols, tid);
   }
-  for (int q = tid; q < B; q += QTHREADS)
-    inv_diag[q] = (q < ncols) ? 1.0f / G[static_cast<size_t>(j0 + q) * d_col + j0 + q] : 0.0f;
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  __syncthreads();
 
-  float w[V], ev[V];
-  const float* wrow = Wk + static_cast<size_t>(rv ? r : 0) * d_col + j0;
+  float* wrow = Ws + rloc * LDG;
+  float* erow = Es + rloc * LDG;
+  if (jp0 >= 0) {
+    // (a) W[rows, blk] -= E_prev[rows] * G[prev blk, blk]  (thread t: chunks t, t+4, ...)
+    constexpr int NCH = B / 16;
+    float4 w4[NCH];
 #pragma unroll
-  for (int c = 0; c < NCH; ++c) {
-    const int col = 16 * c + 4 * t;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (rv && col < ncols) v = *reinterpret_cast<const float4*>(wrow + col);
-    w[4 * c] = v.x; w[4 * c + 1] = v.y; w[4 * c + 2] = v.z; w[4 * c + 3] = v.w;
-    ev[4 * c] = ev[4 * c + 1] = ev[4 * c + 2] = ev[4 * c + 3] = 0.0f;
+    for (int i = 0; i < NCH; ++i) {
+      const int col = 16 * i + 4 * t;
+      w4[i] = (col < ncols) ? *reinterpret_cast<const float4*>(wrow + col)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll 4
+    for (int p = 0; p < B; ++p) {
+      const float e = erow[p];
+      const float* gr = Gs + p * LDG + 4 * t;
+#pragma unroll
+      for (int i = 0; i < NCH; ++i) {
+        if (16 * i + 4 * t >= ncols) continue;
+        const float4 g4 = *reinterpret_cast<const float4*>(gr + 16 * i);
+        w4[i].x = fmaf(-e, g4.x, w4[i].x); w4[i].y = fmaf(-e, g4.y, w4[i].y);
+        w4[i].z = fmaf(-e, g4.z, w4[i].z); w4[i].w = fmaf(-e, g4.w, w4[i].w);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      const int col = 16 * i + 4 * t;
+      if (col < ncols) *reinterpret_cast<float4*>(wrow + col) = w4[i];
+    }
+    __syncthreads();  // every thread is done with the previous block's G rows
+    stage_gblock<B>(Gs, G, d_col, j0, j0, ncols, ncols, tid);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncthreads();
   }
+  for (int q = tid; q < ncols; q += QTHREADS) invd[q] = 1.0f / Gs[q * LDG + q];
 
   const float maxq = static_cast<float>((1 << bits) - 1);
   float s = 1.0f, z = 0.0f;
-  if (GS == 0) {
-    const int g = pc_mode ? 0 : j0 / group;
-    if (!pc_mode && (j0 % group) == 0) {
-      float mn = w[0], mx = w[0];
-#pragma unroll
-      for (int i = 1; i < V; ++i) { mn = fminf(mn, w[i]); mx = fmaxf(mx, w[i]); }
-      const float* rest = Wk + static_cast<size_t>(rv ? r : 0) * d_col;
-      for (int c = j0 + B + t; c < j0 + group; c += 4) {
-        const float v = rest[c];
-        mn = fminf(mn, v); mx = fmaxf(mx, v);
-      }
-      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 2));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      make_params(mn, mx, bits, sym, s, z);
-      if (rv && t == 0) {
-        scales[static_cast<size_t>(r) * n_groups + g] = s;
-        zeros[static_cast<size_t>(r) * n_groups + g] = static_cast<uint8_t>(z);
-      }
-    } else if (rv) {
-      s = scales[static_cast<size_t>(r) * n_groups + g];
-      z = static_cast<float>(zeros[static_cast<size_t>(r) * n_groups + g]);
-    }
+  if (pc_mode) {
+    if (rv) { s = scales[r]; z = static_cast<float>(zeros[r]); }
+  } else if (group > B && (j0 % group) != 0) {  // the group began in an earlier block
+    const int g = j0 / group;
+    if (rv) { s = scales[static_cast<size_t>(r) * n_groups + g];
+              z = static_cast<float>(zeros[static_cast<size_t>(r) * n_groups + g]); }
   }
   __syncthreads();
 
-#pragma unroll
-  for (int q = 0; q < B; ++q) {
-    if (q < ncols) {
-    if (GS != 0 && (q % (GS > 0 ? GS : 1)) == 0) {
+  // (b) 16-column sub-blocks
+  for (int q0 = 0; q0 < ncols; q0 += 16) {
+    if (!pc_mode && ((j0 + q0) % group) == 0) {  // a group starts here
+      const int gend = min(q0 + group, ncols);
       float mn = 3.4e38f, mx = -3.4e38f;
-#pragma unroll
-      for (int c = q / 16; c < (q + (GS > 0 ? GS : 16)) / 16; ++c)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) { mn = fminf(mn, w[4 * c + e]); mx = fmaxf(mx, w[4 * c + e]); }
+      for (int c = q0 + 4 * t; c < gend; c += 16) {
+        const float4 v = *reinterpret_cast<const float4*>(wrow + c);
+        mn = fminf(mn, fminf(fminf(v.x, v.y), fminf(v.z, v.w)));
+        mx = fmaxf(mx, fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
+      }
+      if (group > B && rv) {  // the rest of the group lies right of this block
+        const float* rest = Wk + static_cast<size_t>(r) * d_col;
+        for (int c = j0 + B + t; c < j0 + group; c += 4) {
+          const float v = rest[c];
+          mn = fminf(mn, v); mx = fmaxf(mx, v);
+        }
+      }
       mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
       mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 2));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
       make_params(mn, mx, bits, sym, s, z);
       if (rv && t == 0) {
-        const int g = (j0 + q) / (GS > 0 ? GS : 1);
+        const int g = (j0 + q0) / group;
         scales[static_cast<size_t>(r) * n_groups + g] = s;
         zeros[static_cast<size_t>(r) * n_groups + g] = static_cast<uint8_t>(z);
       }
     }
-    const int tq = (q >> 2) & 3;        // owner thread of column q
-    const int slot = (q >> 4) * 4 + (q & 3);
-    float e = 0.0f;
-    if (t == tq) {
-      const float x = w[slot];
-      float qf = rintf(x / s) + z;
-      qf = fminf(fmaxf(qf, 0.0f), maxq);
-      const float xh = s * (qf - z);
-      e = (x - xh) * inv_diag[q];
-      ev[slot] = e;
-      cstage[rloc * B + q] = static_cast<uint8_t>(qf);
-    }
-    e = __shfl_sync(0xffffffffu, e, qbase | tq);
-    const float* grow = gs + q * B;
+    float4 wv = *reinterpret_cast<const float4*>(wrow + q0 + 4 * t);
+    float w[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
-    for (int c = 0; c < NCH; ++c) {
-      if (16 * c + 15 <= q) continue;  // chunk entirely at or left of q
-      const float4 g4 = *reinterpret_cast<const float4*>(grow + 16 * c + 4 * t);
-      const int kb = 16 * c + 4 * t;
-      if (16 * c > q) {
-        w[4 * c] -= e * g4.x; w[4 * c + 1] -= e * g4.y;
-        w[4 * c + 2] -= e * g4.z; w[4 * c + 3] -= e * g4.w;
-      } else {
-        if (kb > q) w[4 * c] -= e * g4.x;
-        if (kb + 1 > q) w[4 * c + 1] -= e * g4.y;
-        if (kb + 2 > q) w[4 * c + 2] -= e * g4.z;
-        if (kb + 3 > q) w[4 * c + 3] -= e * g4.w;
+    for (int u = 0; u < 16; ++u) {
+      const int q = q0 + u;
+      const int tq = u >> 2;
+      float e = 0.0f;
+      if (t == tq) {
+        const float x = w[u & 3];
+        float qf = rintf(x / s) + z;
+        qf = fminf(fmaxf(qf, 0.0f), maxq);
+        const float xh = s * (qf - z);
+        e = (x - xh) * invd[q];
+        codes[rloc * B + q] = static_cast<uint8_t>(qf);
+        erow[q] = e;
+      }
+      e = __shfl_sync(0xffffffffu, e, qbase | tq);
+      if (u < 15) {
+        const float4 g4 = *reinterpret_cast<const float4*>(Gs + q * LDG + q0 + 4 * t);
+        const int kb = 4 * t;
+        if (kb > u) w[0] = fmaf(-e, g4.x, w[0]);
+        if (kb + 1 > u) w[1] = fmaf(-e, g4.y, w[1]);
+        if (kb + 2 > u) w[2] = fmaf(-e, g4.z, w[2]);
+        if (kb + 3 > u) w[3] = fmaf(-e, g4.w, w[3]);
       }
     }
+    __syncwarp();
+    // rank-16 update of the rest of the block: thread t takes chunks
+    // q0/4 + 4 + t, +4, ... (the chunk it owns in the next sub-block first)
+    if (q0 + 16 < ncols) {
+      float ev[16];
+#pragma unroll
+      for (int u = 0; u < 16; u += 4) {
+        const float4 v = *reinterpret_cast<const float4*>(erow + q0 + u);
+        ev[u] = v.x; ev[u + 1] = v.y; ev[u + 2] = v.z; ev[u + 3] = v.w;
+      }
+      for (int c = q0 + 16 + 4 * t; c < ncols; c += 16) {
+        float4 acc = *reinterpret_cast<const float4*>(wrow + c);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const float4 g4 = *reinterpret_cast<const float4*>(Gs + (q0 + u) * LDG + c);
+          acc.x = fmaf(-ev[u], g4.x, acc.x); acc.y = fmaf(-ev[u], g4.y, acc.y);
+          acc.z = fmaf(-ev[u], g4.z, acc.z); acc.w = fmaf(-ev[u], g4.w, acc.w);
+        }
+        *reinterpret_cast<float4*>(wrow + c) = acc;
+      }
     }
+    __syncwarp();
   }
 
-  // E for the trailing update
+  // (c) E for the trailing update, and the packed codes
   if (rv) {
-    float* erow = E + static_cast<size_t>(r) * B;
-#pragma unroll
-    for (int c = 0; c < NCH; ++c)
-      *reinterpret_cast<float4*>(erow + 16 * c + 4 * t) =
-          make_float4(ev[4 * c], ev[4 * c + 1], ev[4 * c + 2], ev[4 * c + 3]);
-  }
-  __syncwarp();
-  // bit-pack this block's codes: little-endian stream, code k at bits [b k, b k + b)
-  if (rv) {
+    float* eg = Ecur + static_cast<size_t>(r) * B;
+    for (int c = 4 * t; c < B; c += 16)
+      *reinterpret_cast<float4*>(eg + c) = (c < ncols) ? *reinterpret_cast<const float4*>(erow + c)
+                                                       : make_float4(0.f, 0.f, 0.f, 0.f);
     const int nw = ncols * bits / 32;
     const size_t row_words = static_cast<size_t>(d_col) * bits / 32;
     uint32_t* qrow = qweight + static_cast<size_t>(r) * row_words + (static_cast<size_t>(j0) * bits) / 32;
-    const uint8_t* cs = cstage + rloc * B;
+    const uint8_t* cs = codes + rloc * B;
     for (int wi = t; wi < nw; wi += 4) {
       const int bit0 = 32 * wi;
       const int kf = bit0 / bits, kl = (bit0 + 31) / bits;
