@@ -19,6 +19,7 @@
 #include "common.cuh"
 #include "quantize.cuh"
 #include "syrk_tcgen05.cuh"
+#include "trailing_tf32.cuh"
 
 namespace {
 
@@ -109,6 +110,9 @@ gptq_status device_setup(int* num_sms) {
     GPTQ_CUDA_TRY(cudaFuncSetAttribute(quant::block_step_kernel<32>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        quant::block_step_smem<32>()));
+    GPTQ_CUDA_TRY(cudaFuncSetAttribute(trail::trailing_tf32x3_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       trail::SMEM_BYTES));
     GPTQ_CUDA_TRY(cudaStreamCreateWithFlags(&di.aux, cudaStreamNonBlocking));
     for (int i = 0; i < kEvents; ++i)
       GPTQ_CUDA_TRY(cudaEventCreateWithFlags(&di.ev[i], cudaEventDisableTiming));
@@ -160,14 +164,19 @@ PrepareWs prepare_layout(int64_t d) {
 }
 
 struct QuantWs {
-  size_t Wk, E0, E1, total;
+  size_t Wk, E[2][2], Ghi, Glo, total;  // E[buffer][hi/lo]
 };
 QuantWs quant_layout(int64_t d_row, int64_t d_col, int block) {
   QuantWs w{};
   size_t off = 0;
   w.Wk = off; off = align_up(off + static_cast<size_t>(d_row) * d_col * 4);
-  w.E0 = off; off = align_up(off + static_cast<size_t>(d_row) * block * 4);
-  w.E1 = off; off = align_up(off + static_cast<size_t>(d_row) * block * 4);
+  for (int b = 0; b < 2; ++b)
+    for (int h = 0; h < 2; ++h) {
+      w.E[b][h] = off;
+      off = align_up(off + static_cast<size_t>(d_row) * block * 4);
+    }
+  w.Ghi = off; off = align_up(off + static_cast<size_t>(d_col) * d_col * 4);
+  w.Glo = off; off = align_up(off + static_cast<size_t>(d_col) * d_col * 4);
   w.total = off;
   return w;
 }
@@ -183,6 +192,24 @@ CheckWs check_layout(int64_t d_row, int64_t d_col) {
   w.loss = off; off = align_up(off + 8);
   w.total = off;
   return w;
+}
+
+// 2D fp32 tensor map: dims {inner, outer}, row stride in elements, box {bx, by}.
+gptq_status encode_f32_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer,
+                          uint64_t row_stride, uint32_t bx, uint32_t by,
+                          CUtensorMapSwizzle swz) {
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_stride * 4};
+  const cuuint32_t box[2] = {bx, by};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult cr = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(ptr), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) {
+    std::fprintf(stderr, "gptq: cuTensorMapEncodeTiled (f32) failed (%d)\n", static_cast<int>(cr));
+    return GPTQ_ERR_CUDA;
+  }
+  return GPTQ_OK;
 }
 
 // --------------------------------------------------------- SYRK launching
@@ -474,16 +501,39 @@ gptq_status gptq_quantize_layer(const float* W, int64_t d_row, int64_t d_col, co
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* base = static_cast<uint8_t*>(ws);
   float* Wk = reinterpret_cast<float*>(base + L.Wk);
-  float* Ebuf[2] = {reinterpret_cast<float*>(base + L.E0), reinterpret_cast<float*>(base + L.E1)};
+  float* Eb[2][2];
+  for (int b = 0; b < 2; ++b)
+    for (int h = 0; h < 2; ++h) Eb[b][h] = reinterpret_cast<float*>(base + L.E[b][h]);
+  float* Ghi = reinterpret_cast<float*>(base + L.Ghi);
+  float* Glo = reinterpret_cast<float*>(base + L.Glo);
   const int dr = static_cast<int>(d_row), dc = static_cast<int>(d_col);
   const int B = cfg->block, g = cfg->group_size;
   const int n_groups = g ? dc / g : 1;
   const int per_channel = g == 0;
+  int num_sms = 148;
+  st = device_setup(&num_sms);
+  if (st != GPTQ_OK) return st;
+  // tensor maps of the trailing update: E splits (K-major), G splits, W
+  CUtensorMap tm_e[2][2], tm_ghi, tm_glo, tm_w;
+  for (int b = 0; b < 2; ++b)
+    for (int h = 0; h < 2; ++h) {
+      st = encode_f32_2d(&tm_e[b][h], Eb[b][h], B, dr, B, trail::BK, trail::BM,
+                         CU_TENSOR_MAP_SWIZZLE_64B);
+      if (st != GPTQ_OK) return st;
+    }
+  if ((st = encode_f32_2d(&tm_ghi, Ghi, dc, dc, dc, trail::B_BOX, trail::BK,
+                          CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B)) != GPTQ_OK) return st;
+  if ((st = encode_f32_2d(&tm_glo, Glo, dc, dc, dc, trail::B_BOX, trail::BK,
+                          CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B)) != GPTQ_OK) return st;
+  if ((st = encode_f32_2d(&tm_w, Wk, dc, dr, dc, trail::OUT_COLS, trail::BM,
+                          CU_TENSOR_MAP_SWIZZLE_128B)) != GPTQ_OK) return st;
   DeviceInfo* di = current_device_info();
   if (!di) return GPTQ_ERR_CUDA;
 
   quant::prepare_rows_kernel<<<(dr + 7) / 8, 256, 0, s>>>(W, Wk, dead_mask, dr, dc, cfg->bits,
                                                            cfg->sym, per_channel, scales, zeros);
+  GPTQ_LAUNCH_CHECK();
+  trail::split_tf32_kernel<<<4 * num_sms, 256, 0, s>>>(G, Ghi, Glo, static_cast<size_t>(dc) * dc);
   GPTQ_LAUNCH_CHECK();
   // Block j: the step kernel Q_j (caller's stream) applies E_{j-1} to block j
   // and quantizes it; the trailing kernel T_j (auxiliary stream) applies E_j
@@ -504,13 +554,14 @@ gptq_status gptq_quantize_layer(const float* W, int64_t d_row, int64_t d_col, co
     if (jb >= 2 && t_done[jb - 2]) GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, evT[(jb - 2) % 4], 0));
     if (g > B && j0 % g == 0 && jb >= 1 && t_done[jb - 1])  // group params read columns ahead
       GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, evT[(jb - 1) % 4], 0));
-    const float* Ep = jb > 0 ? Ebuf[(jb - 1) & 1] : nullptr;
+    const int pb = (jb - 1) & 1, cb = jb & 1;
+    const float* Eph = jb > 0 ? Eb[pb][0] : nullptr;
+    const float* Epl = jb > 0 ? Eb[pb][1] : nullptr;
     const int jp0 = jb > 0 ? j0 - B : -1;
-    float* Ec = Ebuf[jb & 1];
 #define GPTQ_STEP(BB)                                                                        \
   quant::block_step_kernel<BB><<<qgrid, quant::QTHREADS, quant::block_step_smem<BB>(), s>>>( \
-      Wk, dr, dc, j0, ncols, G, Ep, jp0, Ec, qweight, scales, zeros, cfg->bits, cfg->sym, g,    \
-      n_groups, per_channel)
+      Wk, dr, dc, j0, ncols, G, Eph, Epl, jp0, Eb[cb][0], Eb[cb][1], qweight, scales, zeros,   \
+      cfg->bits, cfg->sym, g, n_groups, per_channel)
     if (B == 128) GPTQ_STEP(128);
     else if (B == 64) GPTQ_STEP(64);
     else GPTQ_STEP(32);
@@ -519,11 +570,15 @@ gptq_status gptq_quantize_layer(const float* W, int64_t d_row, int64_t d_col, co
     GPTQ_CUDA_TRY(cudaEventRecord(evQ[jb % 4], s));
     const int n0 = j0 + 2 * B;  // block jb+1 is updated by Q_{jb+1} itself
     if (n0 < dc) {
-      const int N = dc - n0;
       GPTQ_CUDA_TRY(cudaStreamWaitEvent(di->aux, evQ[jb % 4], 0));
-      const dim3 ugrid((dr + quant::UT - 1) / quant::UT, (N + quant::UT - 1) / quant::UT);
-      quant::trailing_update_kernel<<<ugrid, quant::UTHREADS, 0, di->aux>>>(
-          Wk + n0, Ec, G + static_cast<size_t>(j0) * dc + n0, dr, N, ncols, dc, dc);
+      trail::Params tp{};
+      tp.M = dr; tp.N = dc - n0; tp.K = ncols; tp.n0 = n0; tp.j0 = j0;
+      tp.tiles_m = (dr + trail::BM - 1) / trail::BM;
+      tp.tiles_n = (tp.N + trail::BN - 1) / trail::BN;
+      tp.tiles = tp.tiles_m * tp.tiles_n;
+      const int grid = std::min(tp.tiles, num_sms);
+      trail::trailing_tf32x3_kernel<<<grid, trail::NUM_THREADS, trail::SMEM_BYTES, di->aux>>>(
+          tm_e[cb][0], tm_e[cb][1], tm_ghi, tm_glo, tm_w, tp);
       GPTQ_LAUNCH_CHECK();
       GPTQ_CUDA_TRY(cudaEventRecord(evT[jb % 4], di->aux));
       t_done[jb] = 1;

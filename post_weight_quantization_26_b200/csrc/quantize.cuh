@@ -147,8 +147,9 @@ __device__ __forceinline__ void stage_gblock(float* dst, const float* G, int d_c
 template <int B>
 __global__ void __launch_bounds__(QTHREADS)
 block_step_kernel(const float* __restrict__ Wk, int d_row, int d_col, int j0, int ncols,
-                  const float* __restrict__ G, const float* __restrict__ Eprev, int jp0,
-                  float* __restrict__ Ecur, uint32_t* __restrict__ qweight,
+                  const float* __restrict__ G, const float* __restrict__ Eprev_hi,
+                  const float* __restrict__ Eprev_lo, int jp0, float* __restrict__ Ecur_hi,
+                  float* __restrict__ Ecur_lo, uint32_t* __restrict__ qweight,
                   float* __restrict__ scales, uint8_t* __restrict__ zeros, int bits, int sym,
                   int group, int n_groups, int pc_mode) {
   using L = StepSmem<B>;
@@ -169,7 +170,7 @@ block_step_kernel(const float* __restrict__ Wk, int d_row, int d_col, int j0, in
 
   stage_rows<B>(Ws, Wk + j0, d_col, r0, d_row, ncols, tid);
   if (jp0 >= 0) {
-    stage_rows<B>(Es, Eprev, B, r0, d_row, B, tid);
+    stage_rows<B>(Es, Eprev_hi, B, r0, d_row, B, tid);
     stage_gblock<B>(Gs, G, d_col, jp0, j0, B, ncols, tid);
   } else {
     stage_gblock<B>(Gs, G, d_col, j0, j0, ncols, ncols, tid);
@@ -177,6 +178,19 @@ block_step_kernel(const float* __restrict__ Wk, int d_row, int d_col, int j0, in
   asm volatile("cp.async.commit_group;" ::: "memory");
   asm volatile("cp.async.wait_group 0;" ::: "memory");
   __syncthreads();
+  if (jp0 >= 0) {  // E = E_hi + E_lo (exact): add the low parts in place
+    for (int c = tid; c < QROWS * (B / 4); c += QTHREADS) {
+      const int rr = c / (B / 4), k = (c - rr * (B / 4)) * 4;
+      if (r0 + rr < d_row) {
+        const float4 lo = *reinterpret_cast<const float4*>(Eprev_lo + static_cast<size_t>(r0 + rr) * B + k);
+        float4* hp = reinterpret_cast<float4*>(Es + rr * L::LDG + k);
+        float4 h = *hp;
+        h.x += lo.x; h.y += lo.y; h.z += lo.z; h.w += lo.w;
+        *hp = h;
+      }
+    }
+    __syncthreads();
+  }
 
   float* wrow = Ws + rloc * LDG;
   float* erow = Es + rloc * LDG;
@@ -304,12 +318,21 @@ block_step_kernel(const float* __restrict__ Wk, int d_row, int d_col, int j0, in
     __syncwarp();
   }
 
-  // (c) E for the trailing update, and the packed codes
+  // (c) E for the trailing update as a TF32 split (hi = low 13 mantissa bits
+  // cleared, lo = E - hi), and the packed codes
   if (rv) {
-    float* eg = Ecur + static_cast<size_t>(r) * B;
-    for (int c = 4 * t; c < B; c += 16)
-      *reinterpret_cast<float4*>(eg + c) = (c < ncols) ? *reinterpret_cast<const float4*>(erow + c)
-                                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+    float* eh = Ecur_hi + static_cast<size_t>(r) * B;
+    float* el = Ecur_lo + static_cast<size_t>(r) * B;
+    for (int c = 4 * t; c < B; c += 16) {
+      const float4 v = (c < ncols) ? *reinterpret_cast<const float4*>(erow + c)
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 h = make_float4(__uint_as_float(__float_as_uint(v.x) & 0xFFFFE000u),
+                                   __uint_as_float(__float_as_uint(v.y) & 0xFFFFE000u),
+                                   __uint_as_float(__float_as_uint(v.z) & 0xFFFFE000u),
+                                   __uint_as_float(__float_as_uint(v.w) & 0xFFFFE000u));
+      *reinterpret_cast<float4*>(eh + c) = h;
+      *reinterpret_cast<float4*>(el + c) = make_float4(v.x - h.x, v.y - h.y, v.z - h.z, v.w - h.w);
+    }
     const int nw = ncols * bits / 32;
     const size_t row_words = static_cast<size_t>(d_col) * bits / 32;
     uint32_t* qrow = qweight + static_cast<size_t>(r) * row_words + (static_cast<size_t>(j0) * bits) / 32;

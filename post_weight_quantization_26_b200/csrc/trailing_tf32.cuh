@@ -1,0 +1,256 @@
+// Lazy batched update of the columns right of a block on the 5th-generation
+// tensor cores (dingiv.github.io "量化" page, section GPTQ: after a block of B
+// columns is quantized, all columns to its right are updated at once by one
+// matrix product):
+//     W[:, n0:] -= E * G[j0:j0+K, n0:]
+// E (d_row x K) and G are fp32; the product runs as three TF32 MMAs per
+// K-step on the split operands x = x_hi + x_lo (x_hi = x with the low 13
+// mantissa bits cleared, x_lo = x - x_hi, exact):
+//     E G ~ E_hi G_hi + E_hi G_lo + E_lo G_hi
+// which keeps close to fp32 accuracy (the dropped E_lo G_lo term is ~2^-20
+// of the product).
+//
+// Persistent kernel, 192 threads, tiles of 128 (rows of W) x 256 (columns):
+//   warp 0      TMA producer: per 16-wide K slice, E_hi/E_lo boxes (K-major,
+//               64-byte swizzle) and G_hi/G_lo boxes (MN-major, 128-byte
+//               swizzle with 32-byte atoms, the one MN-major form tf32
+//               operands take), two-deep ring;
+//   warp 1      allocates 256 TMEM columns (one fp32 128x256 accumulator)
+//               and issues tcgen05.mma kind::tf32 from one thread;
+//   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, negate, write a
+//               128x32 tile to shared memory (128-byte swizzle), and add it
+//               into W with a TMA reduce-add (the L2 does the read-modify-
+//               write).
+// Shared memory is kept near 112 KB so a block-step CTA fits on the same SM
+// (the two kernels run concurrently on different streams).  Every mbarrier
+// wait is bounded.
+#pragma once
+
+#include "common.cuh"
+
+namespace gptq {
+namespace trail {
+
+constexpr int BM = 128, BN = 256, BK = 16;
+constexpr int STAGES = 2;
+constexpr int A_BYTES = BM * BK * 4;              // 8 KB (one split)
+constexpr int B_BOX = 32;                          // 32 fp32 = 128 B inner box
+constexpr int B_BOX_BYTES = B_BOX * BK * 4;        // 2 KB
+constexpr int B_BYTES = BN * BK * 4;               // 16 KB (one split)
+constexpr int STAGE_BYTES = 2 * A_BYTES + 2 * B_BYTES;  // 48 KB
+constexpr int OUT_COLS = 32;
+constexpr int OUT_BYTES = BM * OUT_COLS * 4;       // 16 KB
+constexpr int NUM_THREADS = 192;
+constexpr uint32_t TMEM_COLS = 256;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + OUT_BYTES + 1024 + 256;
+
+// kind::tf32 instruction descriptor: fp32 accumulate, A and B tf32 (format
+// 2), A K-major, B MN-major (bit 16), N>>3 at bits 17-22, M>>4 at 24-28.
+constexpr uint32_t IDESC = (1u << 4) | (2u << 7) | (2u << 10) | (1u << 16) |
+                           (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
+
+struct Params {
+  int M;        // rows of W
+  int N;        // columns to update (from n0)
+  int K;        // block width (E and G read as zero past it)
+  int n0;       // first column to update (also the column coordinate into G)
+  int j0;       // first row of G's block
+  int tiles_m, tiles_n, tiles;
+};
+
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo,
+                                              uint32_t layout) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(layout) << 61;
+  return d;
+}
+
+__device__ __forceinline__ void tmem_alloc1(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+               "r"(ncols)
+               : "memory");
+}
+
+__device__ __forceinline__ void named_bar(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+__device__ __forceinline__ void tma_reduce_add_2d(const void* tmap, uint32_t src, int32_t x,
+                                                  int32_t y) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(tmap)),
+      "r"(src), "r"(x), "r"(y)
+      : "memory");
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+trailing_tf32x3_kernel(const __grid_constant__ CUtensorMap tm_ehi,
+                       const __grid_constant__ CUtensorMap tm_elo,
+                       const __grid_constant__ CUtensorMap tm_ghi,
+                       const __grid_constant__ CUtensorMap tm_glo,
+                       const __grid_constant__ CUtensorMap tm_w, const Params p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* base_ptr = smem_raw + (base - raw);
+  const uint32_t ring = base;                                 // STAGES x 48 KB
+  const uint32_t outbuf = base + STAGES * STAGE_BYTES;        // 16 KB, 1024-aligned
+  float* out_ptr = reinterpret_cast<float*>(base_ptr + STAGES * STAGE_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base_ptr + STAGES * STAGE_BYTES + OUT_BYTES);
+  // bars: [0,S) full, [S,2S) empty, 2S tmem_full, 2S+1 tmem_empty
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8u * STAGES;
+  const uint32_t tfull = full0 + 16u * STAGES, tempty = tfull + 8u;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full0 + 8u * s, 1);
+      mbar_init(empty0 + 8u * s, 1);
+    }
+    mbar_init(tfull, 1);
+    mbar_init(tempty, 4);
+    *abort_flag = 0;
+    mbar_fence_init();
+    tma_prefetch_desc(&tm_ehi); tma_prefetch_desc(&tm_elo);
+    tma_prefetch_desc(&tm_ghi); tma_prefetch_desc(&tm_glo); tma_prefetch_desc(&tm_w);
+  }
+  if (warp == 1) {
+    tmem_alloc1(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int nk = (p.K + BK - 1) / BK;  // E is zero past K
+
+  if (warp == 0) {
+    if (lane == 0) {  // ------------------------------------------- producer
+      uint32_t stage = 0, phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.tiles && ok; u += gridDim.x) {
+        const int tm = u % p.tiles_m, tn = u / p.tiles_m;
+        for (int ks = 0; ks < nk; ++ks) {
+          if (!mbar_wait_bounded(empty0 + 8u * stage, phase ^ 1u, abort_flag)) { ok = false; break; }
+          const uint32_t fb = full0 + 8u * stage;
+          mbar_arrive_expect_tx(fb, STAGE_BYTES);
+          const uint32_t s0 = ring + stage * STAGE_BYTES;
+          tma_load_2d(s0, &tm_ehi, fb, ks * BK, tm * BM);
+          tma_load_2d(s0 + A_BYTES, &tm_elo, fb, ks * BK, tm * BM);
+          const int gx = p.n0 + tn * BN, gy = p.j0 + ks * BK;
+#pragma unroll
+          for (int c = 0; c < BN / B_BOX; ++c) {
+            tma_load_2d(s0 + 2 * A_BYTES + c * B_BOX_BYTES, &tm_ghi, fb, gx + c * B_BOX, gy);
+            tma_load_2d(s0 + 2 * A_BYTES + B_BYTES + c * B_BOX_BYTES, &tm_glo, fb, gx + c * B_BOX, gy);
+          }
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {  // ----------------------------------------------- MMA
+      uint32_t stage = 0, phase = 0;
+      int lu = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.tiles && ok; u += gridDim.x, ++lu) {
+        if (!mbar_wait_bounded(tempty, (lu & 1) ^ 1u, abort_flag)) break;
+        tc_fence_after();
+        for (int ks = 0; ks < nk; ++ks) {
+          if (!mbar_wait_bounded(full0 + 8u * stage, phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t s0 = ring + stage * STAGE_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 8; ++kk) {
+            // A: K-major, 64-byte swizzle: 8-row groups 512 B apart; K step = 32 B.
+            const uint64_t ahi = smem_desc(s0 + kk * 32, 16, 512, 4);
+            const uint64_t alo = smem_desc(s0 + A_BYTES + kk * 32, 16, 512, 4);
+            // B: MN-major tf32 takes only the 128-byte swizzle with 32-byte
+            // atoms (4 K-rows of 128 B per atom): 32-column chunks one box
+            // (2 KB) apart, 4-row K groups 512 B apart; this K step's 8 rows
+            // are the kk-th 1 KB slice.
+            const uint64_t bhi = smem_desc(s0 + 2 * A_BYTES + kk * 1024, B_BOX_BYTES, 512, 1);
+            const uint64_t blo = smem_desc(s0 + 2 * A_BYTES + B_BYTES + kk * 1024, B_BOX_BYTES, 512, 1);
+            mma_tf32_ss(tmem_base, ahi, bhi, IDESC, (ks | kk) != 0);
+            mma_tf32_ss(tmem_base, ahi, blo, IDESC, 1);
+            mma_tf32_ss(tmem_base, alo, bhi, IDESC, 1);
+          }
+          mma_commit(empty0 + 8u * stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        mma_commit(tfull);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;  // TMEM lanes [32*quarter, +32) = rows of the tile
+    const int row = quarter * 32 + lane;
+    const bool issuer = (warp == 2 && lane == 0);
+    int lu = 0;
+    for (int u = blockIdx.x; u < p.tiles; u += gridDim.x, ++lu) {
+      const int tm = u % p.tiles_m, tn = u / p.tiles_m;
+      if (!mbar_wait_bounded(tfull, lu & 1, abort_flag)) break;
+      tc_fence_after();
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+      for (int c = 0; c < BN / OUT_COLS; ++c) {
+        if (p.n0 + tn * BN + c * OUT_COLS >= p.n0 + p.N) break;  // past the matrix
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(t_row + c * OUT_COLS, r);
+        tmem_ld_wait();
+        if (issuer) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+        named_bar(1, 128);  // the previous chunk's reduce has read the buffer
+        // 128-byte swizzle: 16-byte chunk j of row r lives at chunk j ^ (r & 7)
+        float* orow = out_ptr + row * OUT_COLS;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int pj = j ^ (row & 7);
+          float4 v = make_float4(-__uint_as_float(r[4 * j]), -__uint_as_float(r[4 * j + 1]),
+                                 -__uint_as_float(r[4 * j + 2]), -__uint_as_float(r[4 * j + 3]));
+          *reinterpret_cast<float4*>(orow + 4 * pj) = v;
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        named_bar(1, 128);
+        if (issuer) {
+          tma_reduce_add_2d(&tm_w, outbuf, p.n0 + tn * BN + c * OUT_COLS, tm * BM);
+          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty);
+    }
+    if (issuer) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// x_hi = x with the low 13 mantissa bits cleared (a TF32 value), x_lo = x - x_hi.
+__global__ void split_tf32_kernel(const float* __restrict__ x, float* __restrict__ hi,
+                                  float* __restrict__ lo, size_t n) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const float v = x[i];
+    const float h = __uint_as_float(__float_as_uint(v) & 0xFFFFE000u);
+    hi[i] = h;
+    lo[i] = v - h;
+  }
+}
+
+}  // namespace trail
+}  // namespace gptq
