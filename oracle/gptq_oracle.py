@@ -54,15 +54,34 @@ def hessian(x_tokens, chunk: int = 16384) -> np.ndarray:
     """``H = 2 * sum_t x_t x_t^T`` in fp64 from token-major ``[n][d]`` input.
 
     bf16 inputs are exact in fp64, and so is each product; only the sum over
-    tokens rounds.  Large inputs are processed ``chunk`` tokens at a time.
+    tokens rounds.  Large inputs are processed ``chunk`` tokens at a time;
+    anything with ``.shape`` whose token slices convert with ``np.asarray``
+    is accepted.
     """
-    x = np.asarray(x_tokens)
+    x = x_tokens if hasattr(x_tokens, "shape") else np.asarray(x_tokens)
     n, d = x.shape
     h = np.zeros((d, d), dtype=F64)
     for t0 in range(0, n, chunk):
         xc = np.asarray(x[t0:t0 + chunk], dtype=F64)
         h += xc.T @ xc
     return 2.0 * h
+
+
+def hessian_rows(x_tokens, rows, chunk: int = 4096) -> np.ndarray:
+    """Rows ``rows`` of ``H = 2 * sum_t x_t x_t^T`` in fp64, for checking a
+    few entries of a Hessian too large to form on the host.
+
+    Same definition as :func:`hessian`, restricted to the requested rows.
+    ``x_tokens`` is token-major ``[n][d]``; it only needs ``.shape`` and
+    slicing along tokens whose slices convert with ``np.asarray``.
+    """
+    rows = np.asarray(rows, dtype=np.int64)
+    n, d = x_tokens.shape
+    out = np.zeros((rows.size, d), dtype=F64)
+    for t0 in range(0, n, chunk):
+        xc = np.asarray(x_tokens[t0:t0 + chunk], dtype=F64)
+        out += xc[:, rows].T @ xc
+    return 2.0 * out
 
 
 # ---------------------------------------------------------------------------

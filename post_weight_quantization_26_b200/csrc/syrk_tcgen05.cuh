@@ -8,15 +8,24 @@
 // split into S chunks so that tiles x chunks fill the 148 SMs evenly; the
 // chunk partials meet in H through fp32 vector atomic adds.
 //
-// Warp roles (192 threads, one CTA per SM, persistent over work units):
+// Accuracy: the tensor cores' fp32 accumulation is not round-to-nearest, and
+// over a long chain of MMAs its error grows with the chain (about 1.5e-4
+// relative after 2300 MMAs, measured against an fp64 sum).  So a TMEM
+// accumulator only ever sums CHAIN_TOKENS tokens from zero; each finished
+// chain is folded into fp32 registers of the epilogue with ordinary
+// round-to-nearest adds, and the chunk's sum leaves through the atomics.
+//
+// Warp roles (320 threads, one CTA per SM, persistent over work units):
 //   warp 0      TMA producer: 64-token stages, A = 2 boxes of 64 features,
 //               B = 4 boxes, 128-byte swizzle, STAGES-deep ring.
 //   warp 1      allocates 512 TMEM columns (two 128x256 fp32 accumulators)
 //               and issues tcgen05.mma (one thread), K = 16 per instruction.
-//   warps 2..5  epilogue: tcgen05.ld the accumulator (each warp its 32-lane
-//               quarter), scale, mask to the upper triangle, atomically add.
-// The accumulator is double-buffered so the epilogue of one unit overlaps
-// the MMAs of the next.  Every mbarrier wait is bounded.
+//   warps 2..9  epilogue: warp w reads TMEM lane quarter (w % 4) and column
+//               half (w - 2) / 4, keeps that 32 x 128 slice of the chunk sum
+//               in registers (128 per thread), and at the end of the unit
+//               scales it, masks it to the upper triangle, and adds it to H.
+// The two TMEM accumulators alternate between chains, so the fold of one
+// chain overlaps the MMAs of the next.  Every mbarrier wait is bounded.
 #pragma once
 
 #include "common.cuh"
@@ -33,7 +42,10 @@ constexpr int BOX_BYTES = BOX * BK * 2;               // 8 KB
 constexpr int A_BYTES = BM * BK * 2;                  // 16 KB
 constexpr int B_BYTES = BN * BK * 2;                  // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;        // 48 KB
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS = 320;
+constexpr int EPI_WARPS = 8;
+constexpr int CHAIN_KB = 8;                           // k-stages per TMEM chain
+constexpr int CHAIN_TOKENS = CHAIN_KB * BK;           // 512 tokens
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 
@@ -105,7 +117,7 @@ syrk_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_x, const Param
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull0 + 8u * a, 1);
-      mbar_init(tempty0 + 8u * a, 4);  // one arrive per epilogue warp
+      mbar_init(tempty0 + 8u * a, EPI_WARPS);  // one arrive per epilogue warp
     }
     *abort_flag = 0;
     mbar_fence_init();
@@ -147,16 +159,20 @@ syrk_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_x, const Param
     // ----------------------------------------------------------------- MMA
     if (lane == 0) {
       uint32_t stage = 0, phase = 0;
-      int lu = 0;
+      uint32_t gc = 0;  // chains issued by this CTA
       bool ok = true;
-      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x, ++lu) {
+      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
         int ti, tj, k0, nk;
         decode_unit(p, u, ti, tj, k0, nk);
-        const uint32_t acc = lu & 1;
-        if (!mbar_wait_bounded(tempty0 + 8u * acc, ((lu >> 1) & 1) ^ 1u, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * BN;
+        uint32_t d_tmem = tmem_base;
         for (int kt = 0; kt < nk; ++kt) {
+          const int kc = kt % CHAIN_KB;
+          if (kc == 0) {  // a new chain starts in the other accumulator
+            const uint32_t acc = gc & 1u;
+            if (!mbar_wait_bounded(tempty0 + 8u * acc, ((gc >> 1) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            d_tmem = tmem_base + acc * BN;
+          }
           if (!mbar_wait_bounded(full0 + 8u * stage, phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = ring + stage * STAGE_BYTES;
@@ -166,56 +182,67 @@ syrk_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_x, const Param
             // 16 tokens = two 8-row core groups of 128 B each = 2048 B.
             const uint64_t ad = smem_desc_sw128(sa + kk * 2048, BOX_BYTES, 1024);
             const uint64_t bd = smem_desc_sw128(sb + kk * 2048, BOX_BYTES, 1024);
-            mma_f16_ss(d_tmem, ad, bd, IDESC, (kt | kk) != 0);
+            mma_f16_ss(d_tmem, ad, bd, IDESC, (kc | kk) != 0);
           }
           mma_commit(empty0 + 8u * stage);  // frees the stage when these MMAs finish
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          if (kc == CHAIN_KB - 1 || kt == nk - 1) {
+            mma_commit(tfull0 + 8u * (gc & 1u));  // chain ready for the fold
+            ++gc;
+          }
         }
-        if (!ok) break;
-        mma_commit(tfull0 + 8u * acc);  // accumulator ready for the epilogue
       }
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter+32)
-    int lu = 0;
-    for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++lu) {
+    const int quarter = warp & 3;          // TMEM lanes [32*quarter, +32)
+    const int half = (warp - 2) >> 2;      // columns [128*half, +128) of the tile
+    uint32_t gc = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
       int ti, tj, k0, nk;
       decode_unit(p, u, ti, tj, k0, nk);
-      const uint32_t acc = lu & 1;
-      if (!mbar_wait_bounded(tfull0 + 8u * acc, (lu >> 1) & 1, abort_flag)) break;
-      tc_fence_after();
-      const int row = ti * BM + quarter * 32 + lane;
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
-      float* hrow = p.H + static_cast<size_t>(row) * p.d;
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(t_row + c * 32, r);
-        tmem_ld_wait();
-        const int jb = tj * BN + c * 32;
-        if (row < p.d && jb + 31 >= row && jb < p.d) {
+      float acc_r[BN / 2];
 #pragma unroll
-          for (int v = 0; v < 8; ++v) {
-            const int j = jb + 4 * v;
-            if (j >= p.d || j + 3 < row) continue;
-            float4 val = make_float4(__uint_as_float(r[4 * v]) * p.scale,
-                                     __uint_as_float(r[4 * v + 1]) * p.scale,
-                                     __uint_as_float(r[4 * v + 2]) * p.scale,
-                                     __uint_as_float(r[4 * v + 3]) * p.scale);
-            if (j >= row) {
-              atomicAdd(reinterpret_cast<float4*>(hrow + j), val);
-            } else {  // the 4-vector straddles the diagonal
-              if (j + 1 >= row) atomicAdd(hrow + j + 1, val.y);
-              if (j + 2 >= row) atomicAdd(hrow + j + 2, val.z);
-              atomicAdd(hrow + j + 3, val.w);
-            }
+      for (int j = 0; j < BN / 2; ++j) acc_r[j] = 0.f;
+      const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+      const int nchains = (nk + CHAIN_KB - 1) / CHAIN_KB;
+      for (int ch = 0; ch < nchains; ++ch, ++gc) {
+        const uint32_t acc = gc & 1u;
+        if (!mbar_wait_bounded(tfull0 + 8u * acc, (gc >> 1) & 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t t0 = tmem_base + lane_off + acc * BN + half * (BN / 2);
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t r[16];
+          tmem_ld_32x32b_x16(t0 + c * 16, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) acc_r[16 * c + j] += __uint_as_float(r[j]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tempty0 + 8u * acc);
+      }
+      if (!ok) break;
+      const int row = ti * BM + quarter * 32 + lane;
+      float* hrow = p.H + static_cast<size_t>(row) * p.d;
+      const int jb0 = tj * BN + half * (BN / 2);
+      if (row < p.d && jb0 + BN / 2 - 1 >= row && jb0 < p.d) {
+#pragma unroll
+        for (int v = 0; v < BN / 8; ++v) {
+          const int j = jb0 + 4 * v;
+          const float4 val = make_float4(acc_r[4 * v] * p.scale, acc_r[4 * v + 1] * p.scale,
+                                         acc_r[4 * v + 2] * p.scale, acc_r[4 * v + 3] * p.scale);
+          if (j < p.d && j >= row) {
+            atomicAdd(reinterpret_cast<float4*>(hrow + j), val);
+          } else if (j < p.d && j + 3 >= row) {  // the 4-vector straddles the diagonal
+            if (j + 1 >= row) atomicAdd(hrow + j + 1, val.y);
+            if (j + 2 >= row) atomicAdd(hrow + j + 2, val.z);
+            atomicAdd(hrow + j + 3, val.w);
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(tempty0 + 8u * acc);
     }
   }
 

@@ -205,7 +205,10 @@ def gen_tokens(spec: LayerSpec, t0: int = 0, t1: int | None = None,
         out[lo - t0: hi - t0].copy_(x[lo - i * CHUNK: hi - i * CHUNK])
 
     chunks = list(range(c0, c1 + 1))
-    nthreads = threads or min(len(chunks), max(1, (os.cpu_count() or 1)))
+    # one chunk's fp32 draws take ~3 x CHUNK x d_col x 4 bytes while in flight
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+    by_mem = max(1, int(12e9 // (3 * CHUNK * spec.d_col * 4)))
+    nthreads = threads or min(len(chunks), max(1, cores), by_mem)
     if nthreads <= 1 or len(chunks) == 1:
         for i in chunks:
             work(i)

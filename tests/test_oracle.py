@@ -127,6 +127,23 @@ def test_hessian_loss_identity():
     assert via_h == pytest.approx(direct, rel=1e-12)
 
 
+def test_hessian_rows_one_hot_and_agreement():
+    """hessian_rows: unit-vector tokens give 2 * counts on the diagonal and
+    zeros elsewhere; on random input it returns exactly the requested rows
+    of the full H (row order kept, repeats allowed)."""
+    d = 7
+    ids = np.array([3, 3, 0, 6, 6, 6, 2, 3])
+    x = np.eye(d)[ids]
+    r = O.hessian_rows(x, [3, 6, 1], chunk=3)
+    want = 2.0 * np.diag(np.bincount(ids, minlength=d))[[3, 6, 1]]
+    np.testing.assert_array_equal(r, want)
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal((1000, 33))
+    rows = [32, 0, 5, 5]
+    np.testing.assert_allclose(O.hessian_rows(x, rows, chunk=128),
+                               O.hessian(x, chunk=256)[rows], rtol=1e-12, atol=1e-9)
+
+
 # ------------------------------------------------------ damping and factor
 def test_dampen_closed_form_and_dead():
     h = np.diag([4.0, 0.0, 8.0])
