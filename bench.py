@@ -197,6 +197,24 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's time: every rank joins one MAX all-reduce (NCCL on
+    the GPUs; any backend whose tensors live on ``device``)."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_value(world: int, d_row: int, d_col: int, ms_max: float) -> float:
+    """Whole-job weights/s: every rank quantizes its own d_row x d_col layer,
+    and the job takes as long as its slowest rank."""
+    return world * d_row * d_col / (ms_max / 1e3)
+
+
 def workload_config(spec, world):
     return {"workload": spec.name, "d_row": spec.d_row, "d_col": spec.d_col,
             "n_tokens": spec.n_tokens, "bits": spec.bits, "group_size": spec.group,
@@ -307,12 +325,8 @@ def run_ours(args, rank, world, local_rank):
     if G.gptq_device_status() != 0:
         raise RuntimeError("device status set during the timed region")
 
-    ms_max = ms
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
-    value = world * dr * d / (ms_max / 1e3)
+    ms_max = max_over_ranks(ms, world, dev)
+    value = weak_value(world, dr, d, ms_max)
 
     # ---- end to end: host buffers in, host buffers out, through the same API
     e2e = None
@@ -418,7 +432,7 @@ def run_e2e(args, G, spec, cfg, x_host, w_host, dev, stream, world):
         zh.copy_(ze, non_blocking=True)
 
     steps = max(1, args.steps)
-    for _ in range(max(1, min(args.warmup, 2))):
+    for _ in range(max(1, min(args.warmup, 3))):
         step()
     torch.cuda.synchronize(dev)
     if world > 1:
@@ -429,14 +443,10 @@ def run_e2e(args, G, spec, cfg, x_host, w_host, dev, stream, world):
         step()
     t1.record(stream)
     torch.cuda.synchronize(dev)
-    ms = t0.elapsed_time(t1) / steps
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(t0.elapsed_time(t1) / steps, world, dev)
     h2d = n * d * 2 + dr * d * 4
     d2h = qw.numel() * 4 + sc.numel() * 4 + ze.numel()
-    return {"value": world * dr * d / (ms / 1e3), "unit": UNIT, "ms_per_step": ms,
+    return {"value": weak_value(world, dr, d, ms), "unit": UNIT, "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
 
