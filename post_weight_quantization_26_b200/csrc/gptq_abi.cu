@@ -237,9 +237,13 @@ void choose_split(int ntiles, int n, int num_sms, int* split_tokens, int* nsplit
 namespace {
 
 // Launch the grouped NT DGEMM with TM-row tiles: persistent CTAs, at most
-// one per SM.  Problems with an empty output are dropped.
+// one per SM, leaving `reserve_sms` SMs free for work that must run beside
+// it (a persistent grid on every SM would keep a later kernel on another
+// stream from starting until it exits).  Problems with an empty output are
+// dropped.
 template <int TM, int WGM>
-gptq_status launch_nt(const std::vector<chol::GemmProblem>& probs, cudaStream_t s) {
+gptq_status launch_nt(const std::vector<chol::GemmProblem>& probs, cudaStream_t s,
+                      int reserve_sms = 0) {
   int num_sms = 148;
   gptq_status st = device_setup(&num_sms);
   if (st != GPTQ_OK) return st;
@@ -256,7 +260,7 @@ gptq_status launch_nt(const std::vector<chol::GemmProblem>& probs, cudaStream_t 
       tiles += q.lower_only ? tm * (tm + 1) / 2 : tm * tn;
     }
     b.tile_start[b.count] = tiles;
-    const int grid = std::min(tiles, num_sms);
+    const int grid = std::min(tiles, std::max(1, num_sms - reserve_sms));
     if (grid > 0) {
       chol::dgemm_nt_kernel<TM, WGM><<<grid, chol::GEMM_THREADS, chol::gemm_smem<TM>(), s>>>(b);
       GPTQ_LAUNCH_CHECK();
@@ -328,6 +332,10 @@ gptq_status gptq_hessian_accumulate(float* H, const void* X, int64_t n, int64_t 
     return GPTQ_ERR_CUDA;
   }
 
+  CUtensorMap tmap_h;  // H as the reduce-add target: 128 rows x 32 fp32 pieces
+  st = encode_f32_2d(&tmap_h, H, d, d, d, syrk::OUT_COLS, syrk::BM, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != GPTQ_OK) return st;
+
   syrk::Params p{};
   p.H = H;
   p.d = static_cast<int>(d);
@@ -343,7 +351,7 @@ gptq_status gptq_hessian_accumulate(float* H, const void* X, int64_t n, int64_t 
   p.units = p.ntiles * p.nsplit;
   const int grid = std::min(p.units, num_sms);
   syrk::syrk_bf16_tcgen05_kernel<<<grid, syrk::NUM_THREADS, syrk::SMEM_BYTES,
-                                   static_cast<cudaStream_t>(stream)>>>(tmap, p);
+                                   static_cast<cudaStream_t>(stream)>>>(tmap, tmap_h, p);
   GPTQ_LAUNCH_CHECK();
   return GPTQ_OK;
 }
@@ -462,7 +470,9 @@ gptq_status gptq_prepare_hinv(const float* H, int64_t d, double damp_rel, float*
       q.M = nk; q.N = rest; q.K = nk; q.alpha = -1.0; q.beta = 0.0;
       uk.push_back(q);
     }
-    st = launch_nt<128, 2>(uk, s);
+    // two SMs stay free for D_k and leaf k+1 on the auxiliary stream (the
+    // leaf's 141 KB of shared memory cannot share an SM with a U_k CTA)
+    st = launch_nt<128, 2>(uk, s, 2);
     if (st != GPTQ_OK) return st;
     GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, evL[k & 1], 0));  // X_{k+1} for P_{k+1}
   }

@@ -6,7 +6,7 @@
 // B(n,k) = X[k][j0+n] come from the same tensor.  Only tiles that touch the
 // upper triangle (i <= j) are computed, 128 x 256 per tile, and tokens are
 // split into S chunks so that tiles x chunks fill the 148 SMs evenly; the
-// chunk partials meet in H through fp32 vector atomic adds.
+// chunk partials meet in H through TMA bulk reduce-adds (fp32 add in L2).
 //
 // Accuracy: the tensor cores' fp32 accumulation is not round-to-nearest, and
 // over a long chain of MMAs its error grows with the chain (about 1.5e-4
@@ -22,8 +22,10 @@
 //               and issues tcgen05.mma (one thread), K = 16 per instruction.
 //   warps 2..9  epilogue: warp w reads TMEM lane quarter (w % 4) and column
 //               half (w - 2) / 4, keeps that 32 x 128 slice of the chunk sum
-//               in registers (128 per thread), and at the end of the unit
-//               scales it, masks it to the upper triangle, and adds it to H.
+//               in registers (128 per thread).  At the end of the unit it
+//               scales the slice, zeroes what lies below the diagonal, and
+//               stages it in 128 x 32 pieces (128-byte swizzle) that one
+//               thread per half adds into H with a TMA reduce-add.
 // The two TMEM accumulators alternate between chains, so the fold of one
 // chain overlaps the MMAs of the next.  Every mbarrier wait is bounded.
 #pragma once
@@ -44,10 +46,13 @@ constexpr int B_BYTES = BN * BK * 2;                  // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;        // 48 KB
 constexpr int NUM_THREADS = 320;
 constexpr int EPI_WARPS = 8;
-constexpr int CHAIN_KB = 8;                           // k-stages per TMEM chain
-constexpr int CHAIN_TOKENS = CHAIN_KB * BK;           // 512 tokens
+constexpr int CHAIN_KB = 16;                          // k-stages per TMEM chain
+constexpr int CHAIN_TOKENS = CHAIN_KB * BK;           // 1024 tokens
+constexpr int OUT_COLS = 32;                          // staged piece: 128 x 32 fp32
+constexpr int OUT_BYTES = BM * OUT_COLS * 4;          // 16 KB, one per column half
 constexpr uint32_t TMEM_COLS = 512;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int SMEM_BYTES =
+    STAGES * STAGE_BYTES + 2 * OUT_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 
 // Instruction descriptor, kind::f16: fp32 accumulate (bits 4-5 = 1), A and B
 // bf16 (bits 7-9 = 1, 10-12 = 1), both MN-major (bits 15, 16), N>>3 at
@@ -92,13 +97,16 @@ __device__ __forceinline__ void decode_unit(const Params& p, int u, int& ti, int
 }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-syrk_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_x, const Params p) {
+syrk_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_x,
+                         const __grid_constant__ CUtensorMap tmap_h, const Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte aligned ring of stages (128B-swizzle atoms are 1024 B).
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t ring = (raw + 1023u) & ~1023u;
   uint8_t* ring_ptr = smem_raw + (ring - raw);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ring_ptr + STAGES * STAGE_BYTES);
+  const uint32_t outbuf0 = ring + STAGES * STAGE_BYTES;  // 2 x 16 KB, 1024-aligned
+  float* out_ptr = reinterpret_cast<float*>(ring_ptr + STAGES * STAGE_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring_ptr + STAGES * STAGE_BYTES + 2 * OUT_BYTES);
   // bars[0..S) full, [S..2S) empty, [2S..2S+2) tmem_full, [2S+2..2S+4) tmem_empty
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -122,6 +130,7 @@ syrk_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_x, const Param
     *abort_flag = 0;
     mbar_fence_init();
     tma_prefetch_desc(&tmap_x);
+    tma_prefetch_desc(&tmap_h);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
@@ -197,9 +206,12 @@ syrk_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_x, const Param
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;          // TMEM lanes [32*quarter, +32)
     const int half = (warp - 2) >> 2;      // columns [128*half, +128) of the tile
+    // The eight epilogue warps meet at named barriers, so their control flow
+    // stays uniform even after a wait gives up: a warp that timed out keeps
+    // looping (skipping the work) instead of leaving the others waiting.
     uint32_t gc = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+    for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
       int ti, tj, k0, nk;
       decode_unit(p, u, ti, tj, k0, nk);
       float acc_r[BN / 2];
@@ -209,7 +221,8 @@ syrk_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_x, const Param
       const int nchains = (nk + CHAIN_KB - 1) / CHAIN_KB;
       for (int ch = 0; ch < nchains; ++ch, ++gc) {
         const uint32_t acc = gc & 1u;
-        if (!mbar_wait_bounded(tfull0 + 8u * acc, (gc >> 1) & 1u, abort_flag)) { ok = false; break; }
+        if (ok && !mbar_wait_bounded(tfull0 + 8u * acc, (gc >> 1) & 1u, abort_flag)) ok = false;
+        if (!ok) continue;
         tc_fence_after();
         const uint32_t t0 = tmem_base + lane_off + acc * BN + half * (BN / 2);
 #pragma unroll
@@ -224,26 +237,40 @@ syrk_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_x, const Param
         __syncwarp();
         if (lane == 0) mbar_arrive(tempty0 + 8u * acc);
       }
-      if (!ok) break;
-      const int row = ti * BM + quarter * 32 + lane;
-      float* hrow = p.H + static_cast<size_t>(row) * p.d;
-      const int jb0 = tj * BN + half * (BN / 2);
-      if (row < p.d && jb0 + BN / 2 - 1 >= row && jb0 < p.d) {
+      // scale, mask to the upper triangle, stage, and reduce-add into H
+      const int rl = quarter * 32 + lane;           // row within the tile
+      const int row = ti * BM + rl;
+      const bool issuer = lane == 0 && quarter == 2;  // warps 2 and 6
+      float* orow = out_ptr + half * (OUT_BYTES / 4) + rl * OUT_COLS;
 #pragma unroll
-        for (int v = 0; v < BN / 8; ++v) {
-          const int j = jb0 + 4 * v;
-          const float4 val = make_float4(acc_r[4 * v] * p.scale, acc_r[4 * v + 1] * p.scale,
-                                         acc_r[4 * v + 2] * p.scale, acc_r[4 * v + 3] * p.scale);
-          if (j < p.d && j >= row) {
-            atomicAdd(reinterpret_cast<float4*>(hrow + j), val);
-          } else if (j < p.d && j + 3 >= row) {  // the 4-vector straddles the diagonal
-            if (j + 1 >= row) atomicAdd(hrow + j + 1, val.y);
-            if (j + 2 >= row) atomicAdd(hrow + j + 2, val.z);
-            atomicAdd(hrow + j + 3, val.w);
+      for (int c = 0; c < BN / 2 / OUT_COLS; ++c) {
+        const int x0 = tj * BN + half * (BN / 2) + c * OUT_COLS;  // first column of the piece
+        // pieces past the matrix or wholly below the diagonal add nothing
+        const bool live = ok && x0 < p.d && x0 + OUT_COLS - 1 >= ti * BM;
+        if (issuer) bulk_wait_read0();   // this half's previous piece has left the buffer
+        named_bar(1, 32 * EPI_WARPS);
+        if (live) {
+#pragma unroll
+          for (int q = 0; q < OUT_COLS / 4; ++q) {
+            const int j = x0 + 4 * q;
+            float4 v;
+            v.x = (j >= row) ? acc_r[c * OUT_COLS + 4 * q] * p.scale : 0.f;
+            v.y = (j + 1 >= row) ? acc_r[c * OUT_COLS + 4 * q + 1] * p.scale : 0.f;
+            v.z = (j + 2 >= row) ? acc_r[c * OUT_COLS + 4 * q + 2] * p.scale : 0.f;
+            v.w = (j + 3 >= row) ? acc_r[c * OUT_COLS + 4 * q + 3] * p.scale : 0.f;
+            // 128-byte swizzle: 16-byte chunk q of row r sits at chunk q ^ (r & 7)
+            *reinterpret_cast<float4*>(orow + 4 * (q ^ (rl & 7))) = v;
           }
+          fence_proxy_async_smem();
+        }
+        named_bar(1, 32 * EPI_WARPS);
+        if (issuer && live) {
+          tma_reduce_add_2d(&tmap_h, outbuf0 + half * OUT_BYTES, x0, ti * BM);
+          bulk_commit();
         }
       }
     }
+    if (lane == 0 && quarter == 2) bulk_wait0();  // the reduce-adds have landed in H
   }
 
   tc_fence_before();

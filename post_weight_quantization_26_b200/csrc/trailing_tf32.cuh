@@ -15,8 +15,10 @@
 //               64-byte swizzle) and G_hi/G_lo boxes (MN-major, 128-byte
 //               swizzle with 32-byte atoms, the one MN-major form tf32
 //               operands take), two-deep ring;
-//   warp 1      allocates 256 TMEM columns (one fp32 128x256 accumulator)
-//               and issues tcgen05.mma kind::tf32 from one thread;
+//   warp 1      allocates 512 TMEM columns (two fp32 128x256 accumulators,
+//               used by alternate tiles so that one tile's epilogue overlaps
+//               the next tile's MMAs) and issues tcgen05.mma kind::tf32 from
+//               one thread;
 //   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, negate, write a
 //               128x32 tile to shared memory (128-byte swizzle), and add it
 //               into W with a TMA reduce-add (the L2 does the read-modify-
@@ -41,7 +43,7 @@ constexpr int STAGE_BYTES = 2 * A_BYTES + 2 * B_BYTES;  // 48 KB
 constexpr int OUT_COLS = 32;
 constexpr int OUT_BYTES = BM * OUT_COLS * 4;       // 16 KB
 constexpr int NUM_THREADS = 192;
-constexpr uint32_t TMEM_COLS = 256;
+constexpr uint32_t TMEM_COLS = 512;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + OUT_BYTES + 1024 + 256;
 
 // kind::tf32 instruction descriptor: fp32 accumulate, A and B tf32 (format
@@ -75,19 +77,6 @@ __device__ __forceinline__ void tmem_alloc1(uint32_t dst_smem, uint32_t ncols) {
                : "memory");
 }
 
-__device__ __forceinline__ void named_bar(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
-__device__ __forceinline__ void tma_reduce_add_2d(const void* tmap, uint32_t src, int32_t x,
-                                                  int32_t y) {
-  asm volatile(
-      "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-          reinterpret_cast<uint64_t>(tmap)),
-      "r"(src), "r"(x), "r"(y)
-      : "memory");
-}
-
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 trailing_tf32x3_kernel(const __grid_constant__ CUtensorMap tm_ehi,
                        const __grid_constant__ CUtensorMap tm_elo,
@@ -102,21 +91,23 @@ trailing_tf32x3_kernel(const __grid_constant__ CUtensorMap tm_ehi,
   const uint32_t outbuf = base + STAGES * STAGE_BYTES;        // 16 KB, 1024-aligned
   float* out_ptr = reinterpret_cast<float*>(base_ptr + STAGES * STAGE_BYTES);
   uint64_t* bars = reinterpret_cast<uint64_t*>(base_ptr + STAGES * STAGE_BYTES + OUT_BYTES);
-  // bars: [0,S) full, [S,2S) empty, 2S tmem_full, 2S+1 tmem_empty
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 2);
+  // bars: [0,S) full, [S,2S) empty, [2S,2S+2) tmem_full, [2S+2,2S+4) tmem_empty
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8u * STAGES;
-  const uint32_t tfull = full0 + 16u * STAGES, tempty = tfull + 8u;
+  const uint32_t tfull0 = full0 + 16u * STAGES, tempty0 = tfull0 + 16u;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full0 + 8u * s, 1);
       mbar_init(empty0 + 8u * s, 1);
     }
-    mbar_init(tfull, 1);
-    mbar_init(tempty, 4);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull0 + 8u * a, 1);
+      mbar_init(tempty0 + 8u * a, 4);  // one arrive per epilogue warp
+    }
     *abort_flag = 0;
     mbar_fence_init();
     tma_prefetch_desc(&tm_ehi); tma_prefetch_desc(&tm_elo);
@@ -162,8 +153,10 @@ trailing_tf32x3_kernel(const __grid_constant__ CUtensorMap tm_ehi,
       int lu = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < p.tiles && ok; u += gridDim.x, ++lu) {
-        if (!mbar_wait_bounded(tempty, (lu & 1) ^ 1u, abort_flag)) break;
+        const uint32_t acc = lu & 1;
+        if (!mbar_wait_bounded(tempty0 + 8u * acc, ((lu >> 1) & 1) ^ 1u, abort_flag)) break;
         tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
         for (int ks = 0; ks < nk; ++ks) {
           if (!mbar_wait_bounded(full0 + 8u * stage, phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
@@ -179,15 +172,15 @@ trailing_tf32x3_kernel(const __grid_constant__ CUtensorMap tm_ehi,
             // are the kk-th 1 KB slice.
             const uint64_t bhi = smem_desc(s0 + 2 * A_BYTES + kk * 1024, B_BOX_BYTES, 512, 1);
             const uint64_t blo = smem_desc(s0 + 2 * A_BYTES + B_BYTES + kk * 1024, B_BOX_BYTES, 512, 1);
-            mma_tf32_ss(tmem_base, ahi, bhi, IDESC, (ks | kk) != 0);
-            mma_tf32_ss(tmem_base, ahi, blo, IDESC, 1);
-            mma_tf32_ss(tmem_base, alo, bhi, IDESC, 1);
+            mma_tf32_ss(d_tmem, ahi, bhi, IDESC, (ks | kk) != 0);
+            mma_tf32_ss(d_tmem, ahi, blo, IDESC, 1);
+            mma_tf32_ss(d_tmem, alo, bhi, IDESC, 1);
           }
           mma_commit(empty0 + 8u * stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        mma_commit(tfull);
+        mma_commit(tfull0 + 8u * acc);
       }
     }
     __syncwarp();
@@ -196,18 +189,28 @@ trailing_tf32x3_kernel(const __grid_constant__ CUtensorMap tm_ehi,
     const int quarter = warp & 3;  // TMEM lanes [32*quarter, +32) = rows of the tile
     const int row = quarter * 32 + lane;
     const bool issuer = (warp == 2 && lane == 0);
+    // The four epilogue warps meet at named barriers, so a warp whose wait
+    // gave up keeps looping (skipping the work) rather than leave the others
+    // waiting at a barrier it will not reach.
+    bool ok = true;
     int lu = 0;
     for (int u = blockIdx.x; u < p.tiles; u += gridDim.x, ++lu) {
       const int tm = u % p.tiles_m, tn = u / p.tiles_m;
-      if (!mbar_wait_bounded(tfull, lu & 1, abort_flag)) break;
+      const uint32_t acc = lu & 1;
+      if (ok && !mbar_wait_bounded(tfull0 + 8u * acc, (lu >> 1) & 1, abort_flag)) ok = false;
       tc_fence_after();
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
       for (int c = 0; c < BN / OUT_COLS; ++c) {
         if (p.n0 + tn * BN + c * OUT_COLS >= p.n0 + p.N) break;  // past the matrix
         uint32_t r[32];
-        tmem_ld_32x32b_x32(t_row + c * OUT_COLS, r);
-        tmem_ld_wait();
-        if (issuer) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+        if (ok) {
+          tmem_ld_32x32b_x32(t_row + c * OUT_COLS, r);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) r[j] = 0u;
+        }
+        if (issuer) bulk_wait_read0();
         named_bar(1, 128);  // the previous chunk's reduce has read the buffer
         // 128-byte swizzle: 16-byte chunk j of row r lives at chunk j ^ (r & 7)
         float* orow = out_ptr + row * OUT_COLS;
@@ -218,18 +221,18 @@ trailing_tf32x3_kernel(const __grid_constant__ CUtensorMap tm_ehi,
                                  -__uint_as_float(r[4 * j + 2]), -__uint_as_float(r[4 * j + 3]));
           *reinterpret_cast<float4*>(orow + 4 * pj) = v;
         }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        fence_proxy_async_smem();
         named_bar(1, 128);
-        if (issuer) {
+        if (issuer && ok) {
           tma_reduce_add_2d(&tm_w, outbuf, p.n0 + tn * BN + c * OUT_COLS, tm * BM);
-          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+          bulk_commit();
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(tempty);
+      if (lane == 0) mbar_arrive(tempty0 + 8u * acc);
     }
-    if (issuer) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    if (issuer) bulk_wait0();
   }
 
   tc_fence_before();
