@@ -94,69 +94,34 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 
 // ------------------------------------------------------------------ leaf
 // Factor the n x n (n <= NB, n % 8 == 0) diagonal block at A (leading dim
-// lda) and write X = L^-1: row-major to Xout (NB x NB, zero above the
-// diagonal) and transposed to Mt (leading dim ldm; zero below the diagonal
-// there).  One CTA of 32 warps; the lower triangle is cut into 4x4 tiles
-// held in registers: warp w owns tile row w and lane l the tile in column l
-// (lanes right of the diagonal idle), which keeps the per-step code small
-// enough to stay in the instruction cache.  The sweep takes 4 columns per
-// step J:
-//   1. the step's 4x4 diagonal tile was handed over by its owner and
-//      factored once into X4 = chol(D)^-1;
-//   2. lane J's tiles below the diagonal form L = A X4^T (and then hold M,
-//      starting from 0); row J's tiles left of it rescale M_J <- X4 M_J; all
-//      of these go to Vt (V transposed, 4 x NB);
-//   3. every tile below the step does t -= V_i V_x^T: the row operand is one
-//      broadcast per warp, the column operand a contiguous per-lane read.
-//      The owner of the next diagonal tile updates and factors it first.
-// Each position holds A's value until its columns are eliminated and M's
-// value afterwards, so one sweep yields M = L^-1.  A non-positive or
-// non-finite pivot records the original-order column d-1-(gcol0+j) in
-// *bad_pivot (first failure only) and the sweep goes on.
-constexpr int LEAF_THREADS = 1024;  // 32 warps: one tile row each
-constexpr int LSLOTS = 1;
-constexpr int TS = NB + 2;   // staging row stride (doubles)
-
-// In place on a 4x4 tile (row-major, lower part read): Cholesky D = L4 L4^T,
-// then L4 -> X4 = L4^-1 (lower, upper part zeroed).  Row i of X is formed
-// left to right, so each l_ij is read before it is overwritten.
-__device__ __forceinline__ void chol_inv4_inplace(double (&a)[16], int col0, int d,
-                                                  long long* bad_pivot) {
-  double iv[4];
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    double p = a[5 * c];
-#pragma unroll
-    for (int k = 0; k < c; ++k) p = fma(-a[4 * c + k], a[4 * c + k], p);
-    if (!(p > 0.0 && isfinite(p)))
-      atomicCAS(reinterpret_cast<unsigned long long*>(bad_pivot),
-                static_cast<unsigned long long>(-1ll),
-                static_cast<unsigned long long>(d - 1 - (col0 + c)));
-    iv[c] = rsqrt(p);
-    a[5 * c] = p * iv[c];
-#pragma unroll
-    for (int i = c + 1; i < 4; ++i) {
-      double t = a[4 * i + c];
-#pragma unroll
-      for (int k = 0; k < c; ++k) t = fma(-a[4 * i + k], a[4 * c + k], t);
-      a[4 * i + c] = t * iv[c];
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-#pragma unroll
-    for (int j = 0; j < i; ++j) {
-      double t = 0.0;  // sum_{k=j}^{i-1} l_ik x_kj  (x_jj = iv[j], rows k < i already X)
-#pragma unroll
-      for (int k = j; k < i; ++k) t = fma(a[4 * i + k], (k == j) ? iv[j] : a[4 * k + j], t);
-      a[4 * i + j] = -iv[i] * t;
-    }
-#pragma unroll
-    for (int j = i + 1; j < 4; ++j) a[4 * i + j] = 0.0;
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) a[5 * i] = iv[i];
-}
+// d) and form X = L^-1.  Output: X row-major to Xout (NB x NB, zero above
+// the diagonal, identity past n) and X^T into the block of Mt (leading dim
+// d; zero below the diagonal there).
+//
+// One CTA of 8 warps keeps the whole block in shared memory S (identity past
+// n, zero above the diagonal).  With the block cut into 16 x 16 blocks
+// (i, j), the sweep takes the 16-column panels p = 0..7:
+//   (i)   one warp factors the diagonal block A_pp = L_pp L_pp^T in
+//         registers (lane = row; pivots and L entries travel by shuffle)
+//         and inverts it, X_pp = L_pp^-1 (lane = column), into Xd[p];
+//   (ii)  L_ip = A_ip X_pp^T for the blocks below the diagonal block, and
+//         X_pj = X_pp R_pj for the blocks left of it (one warp per block);
+//   (iii) A_ik -= L_ip L_kp^T for p < k <= i, and R_ij -= L_ip X_pj for
+//         i > p, j <= p.  R_ij starts at 0 and collects -sum_{k<p} L_ik X_kj,
+//         so X_ij = X_ii R_ij once panel i is reached (block forward
+//         substitution on the identity).
+// R_ij, and then X_ij, live transposed in S's strict upper blocks (block
+// (j, i)), which is the layout of X^T that Mt wants.  Steps (ii) and (iii)
+// run on the fp64 MMA (m8n8k4), one 16 x 16 block per warp job.  In (iii)
+// warp 0 updates the next diagonal block first and factors it while the
+// other warps finish the rest, so the serial part overlaps the updates.
+// Two barriers per panel.  A non-positive or non-finite pivot records the
+// original-order column d-1-(gcol0+j) in *bad_pivot (first failure only)
+// and the sweep goes on.
+constexpr int LEAF_THREADS = 256;
+constexpr int LS = NB + 4;       // S row stride (doubles): fragment loads in two wavefronts
+constexpr int XDS = 20;          // Xd row stride (doubles)
+constexpr int LEAF_SMEM = (NB * LS + 8 * 16 * XDS) * 8;
 
 __device__ __forceinline__ void dmma_8x8x4(double& c0, double& c1, double a, double b) {
   asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
@@ -164,189 +129,303 @@ __device__ __forceinline__ void dmma_8x8x4(double& c0, double& c1, double a, dou
                : "d"(a), "d"(b));
 }
 
-__device__ __forceinline__ int leaf_tile_row(int warp, int /*s*/) { return warp; }
-
-__device__ void leaf_factor_invert(const double* __restrict__ A, long long lda, int n,
-                                   double* __restrict__ Xout, double* __restrict__ Mt,
-                                   long long ldm, long long* __restrict__ bad_pivot, int gcol0,
-                                   int d, double* __restrict__ sm) {
-  double* Vt = sm;             // 4 x NB
-  double* Xs = Vt + 4 * NB;    // X4 of the current step
-  double* Dg = Xs + 16;        // the next diagonal tile, handed to its factorization
-  double* T = Dg + 16;         // NB x TS staging of the whole block
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  {  // the block's rows into shared memory, 16-byte chunks in flight at once
-    const int cpr = n / 2;
-    for (int c = tid; c < n * cpr; c += LEAF_THREADS) {
-      const int i = c / cpr, x = (c - i * cpr) * 2;
-      cp_async16(smem_u32(T + i * TS + x), A + static_cast<long long>(i) * lda + x, 16);
-    }
-    cp_async_commit();
-    cp_async_wait<0>();
-  }
-  __syncthreads();
-  const int nt = n / 4;  // tile rows/columns in use
-  double r[LSLOTS][16];
+// 16 x 16 x 16 block product on one warp, acc += A B, with A(r, q) and
+// B(q, c) given by accessors.  acc[rt][ct][e] is the m8n8 fragment element
+// (8 rt + lane/4, 8 ct + 2 (lane%4) + e).
+template <class FA, class FB>
+__device__ __forceinline__ void blk16_mma(double (&acc)[2][2][2], FA fa, FB fb, int lane) {
+  const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-  for (int s = 0; s < LSLOTS; ++s) {
-    const int bi = leaf_tile_row(warp, s);
-#pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const int i = 4 * bi + (e >> 2), x = 4 * lane + (e & 3);
-      r[s][e] = (bi < nt && x <= i) ? T[i * TS + x] : 0.0;
-    }
-  }
-  // the 4x4 diagonal tile at (j, j) went to Dg; factor it once into Xs
-  auto factor_diag = [&](int j) {
-    double t[16];
-#pragma unroll
-    for (int e = 0; e < 16; ++e) t[e] = Dg[e];
-    chol_inv4_inplace(t, gcol0 + 4 * j, d, bad_pivot);
-#pragma unroll
-    for (int e = 0; e < 16; ++e) Xs[e] = t[e];
-  };
-  if (warp == 0 && lane == 0) {  // step 0's diagonal tile is final already
-#pragma unroll
-    for (int e = 0; e < 16; ++e) Dg[e] = r[0][e];
-    factor_diag(0);
-  }
-  double* Cs = T + NB * TS;   // raw column-block values of the step, NB x 4
-  for (int J = 0; J < nt; ++J) {
-    __syncthreads();  // X4 of step J is in Xs; the last update's reads of Vt are done
-    const double* X4 = Xs;  // read through shared memory (a broadcast) to save registers
-    // (warp-uniform branches; lane J's tile travels by shuffle)
-    constexpr unsigned FULL = 0xffffffffu;
-#pragma unroll
-    for (int s = 0; s < LSLOTS; ++s) {
-      const int bi = leaf_tile_row(warp, s);
-      if (bi >= nt) continue;
-      if (bi > J) {  // stage lane J's raw values (column block J); M starts at 0 there
-        double mine = 0.0;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const double v = __shfl_sync(FULL, r[s][e], J);
-          if (lane == e) mine = v;
-        }
-        if (lane < 16) Cs[(4 * bi + (lane >> 2)) * 4 + (lane & 3)] = mine;
-        const bool z = lane == J;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) r[s][e] = z ? 0.0 : r[s][e];
-      } else if (bi == J) {  // the diagonal tile becomes X4; row block J: M_J <- X4 M_J
-        double m[16];
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            double t = 0.0;
-#pragma unroll
-            for (int bb = 0; bb <= a; ++bb) t = fma(X4[4 * a + bb], r[s][4 * bb + c], t);
-            m[4 * a + c] = t;
-          }
-        const bool diag = lane == J, left = lane < J;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) r[s][e] = diag ? X4[e] : (left ? m[e] : r[s][e]);
-        if (lane <= J) {
-#pragma unroll
-          for (int a = 0; a < 4; ++a)
-#pragma unroll
-            for (int c = 0; c < 4; ++c) Vt[a * NB + 4 * lane + c] = r[s][4 * a + c];
-        }
-      }
-    }
-    __syncthreads();  // the step's column block is staged
-    // L = A X4^T for every row below the step: two outputs per thread
-    for (int o = tid; o < 2 * n; o += LEAF_THREADS) {
-      const int i = o >> 1, c0 = 2 * (o & 1);
-      if (i <= 4 * J + 3) continue;
-      const double2 ra = *reinterpret_cast<const double2*>(Cs + i * 4);
-      const double2 rb = *reinterpret_cast<const double2*>(Cs + i * 4 + 2);
-      auto lrow = [&](int c, double x0, double x1, double x2, double x3) {
-        double t = ra.x * x0;
-        t = fma(ra.y, x1, t);
-        t = fma(rb.x, x2, t);
-        t = fma(rb.y, x3, t);
-        Vt[c * NB + i] = t;
-      };
-      if (c0 == 0) {
-        lrow(0, X4[0], X4[1], X4[2], X4[3]);
-        lrow(1, X4[4], X4[5], X4[6], X4[7]);
-      } else {
-        lrow(2, X4[8], X4[9], X4[10], X4[11]);
-        lrow(3, X4[12], X4[13], X4[14], X4[15]);
-      }
-    }
-    __syncthreads();  // Vt is complete
-    // t -= V_i V_x^T for every tile row below the step.  The owner of the
-    // next diagonal tile hands it over (Dg) and factors it after its rows.
-    const int Jn = J + 1;
-    bool owner = false;
-#pragma unroll
-    for (int s = 0; s < LSLOTS; ++s) {
-      const int bi = leaf_tile_row(warp, s);
-      if (bi >= nt || bi <= J) continue;
-#pragma unroll
-      for (int bb = 0; bb < 4; ++bb) {
-        const double2* pv = reinterpret_cast<const double2*>(Vt + bb * NB + 4 * bi);
-        const double2* px = reinterpret_cast<const double2*>(Vt + bb * NB + 4 * lane);
-        const double2 v0 = pv[0], v1 = pv[1], x0 = px[0], x1 = px[1];
-        const double vi[4] = {v0.x, v0.y, v1.x, v1.y};
-        const double vx[4] = {x0.x, x0.y, x1.x, x1.y};
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-          for (int c = 0; c < 4; ++c) r[s][4 * a + c] = fma(-vi[a], vx[c], r[s][4 * a + c]);
-      }
-      if (bi == Jn && lane == Jn) {
-        owner = true;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) Dg[e] = r[s][e];
-      }
-    }
-    if (owner) factor_diag(Jn);
-  }
-  __syncthreads();  // everyone is done with T's input values
-#pragma unroll
-  for (int s = 0; s < LSLOTS; ++s) {
-    const int bi = leaf_tile_row(warp, s);
-    if (bi >= nt || lane > bi) continue;
-#pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const int i = 4 * bi + (e >> 2), x = 4 * lane + (e & 3);
-      if (x <= i) T[i * TS + x] = r[s][e];
-    }
-  }
-  __syncthreads();
-  // coalesced writes: X row-major (zero above), M^T into the diagonal block
-  for (int idx = tid; idx < NB * NB / 2; idx += LEAF_THREADS) {
-    const int i = (2 * idx) / NB, x = 2 * idx - i * NB;
-    const double v0 = (x <= i && i < n) ? T[i * TS + x] : 0.0;
-    const double v1 = (x + 1 <= i && i < n) ? T[i * TS + x + 1] : 0.0;
-    reinterpret_cast<double2*>(Xout)[idx] = make_double2(v0, v1);
-  }
-  for (int idx = tid; idx < n * n; idx += LEAF_THREADS) {
-    const int row = idx / n, col = idx - row * n;  // Mt[row][col] = M[col][row]
-    Mt[static_cast<long long>(row) * ldm + col] = (row <= col) ? T[col * TS + row] : 0.0;
+  for (int k4 = 0; k4 < 4; ++k4) {
+    const double a0 = fa(g, 4 * k4 + t), a1 = fa(8 + g, 4 * k4 + t);
+    const double b0 = fb(4 * k4 + t, g), b1 = fb(4 * k4 + t, 8 + g);
+    dmma_8x8x4(acc[0][0][0], acc[0][0][1], a0, b0);
+    dmma_8x8x4(acc[0][1][0], acc[0][1][1], a0, b1);
+    dmma_8x8x4(acc[1][0][0], acc[1][0][1], a1, b0);
+    dmma_8x8x4(acc[1][1][0], acc[1][1][1], a1, b1);
   }
 }
 
-// One CTA factors the diagonal block at (off, off) of A: X -> Xout, M^T -> Mt.
+// (i) on one warp: factor the diagonal block p of S, A_pp = L_pp L_pp^T, and
+// write X_pp = L_pp^-1 row-major (stride XDS, zero above the diagonal) to
+// Xd[p].  Lane c holds column c of the block in registers (lanes 16..31
+// shadow lanes 0..15), unscaled during the sweep.  At pivot j every lane
+// receives the pivot and column j by shuffle (issued together) and scales
+// what it receives by 1/sqrt(pivot); lane c > j then updates its column,
+// a_ic -= l_ij l_cj.  The serial chain per pivot is one shuffle, rsqrt, one
+// multiply and one FMA.  After the sweep each lane scales its own column
+// once.  Branch-free; a bad pivot is reported once, after the sweep.
+__device__ __noinline__ void leaf_diag_factor(const double* __restrict__ S,
+                                              double* __restrict__ Xd, int p, int n,
+                                              int gcol0, int d, long long* bad_pivot,
+                                              int lane) {
+  constexpr unsigned FULL = 0xffffffffu;
+  const int c0 = 16 * p, c = lane & 15;
+  const double* D = S + c0 * LS + c0;
+  double col[16], rme = 0.0;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) col[i] = (i >= c) ? D[i * LS + c] : 0.0;
+  unsigned badmask = 0u;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    double aij[16];
+    const double piv = __shfl_sync(FULL, col[j], j);
+#pragma unroll
+    for (int i = j + 1; i < 16; ++i) aij[i] = __shfl_sync(FULL, col[i], j);
+    badmask |= (piv > 0.0 && isfinite(piv)) ? 0u : (1u << j);
+    const double r = rsqrt(piv);
+    rme = (c == j) ? r : rme;
+    // l_cj becomes known at i == c; rows above c see l_cj = 0 and stay put
+    double lcj = 0.0;
+#pragma unroll
+    for (int i = j + 1; i < 16; ++i) {
+      const double lij = aij[i] * r;
+      lcj = (c == i) ? lij : lcj;
+      col[i] = fma(-lij, lcj, col[i]);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) col[i] = (i >= c) ? col[i] * rme : 0.0;  // L's column c
+  // column c of X = L^-1: x_kc = -(sum_{m<k} l_km x_mc) / l_kk, right-looking
+  double x[16], acc[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) acc[k] = 0.0;
+#pragma unroll
+  for (int m = 0; m < 16; ++m) {
+    // row entries l_km (k > m) from lane m, fetched before x_m is needed
+    double lkm[16];
+#pragma unroll
+    for (int k = m + 1; k < 16; ++k) lkm[k] = __shfl_sync(FULL, col[k], m);
+    const double rm = __shfl_sync(FULL, rme, m);
+    x[m] = (m == c) ? rm : ((m > c) ? -acc[m] * rm : 0.0);
+#pragma unroll
+    for (int k = m + 1; k < 16; ++k) acc[k] = fma(lkm[k], x[m], acc[k]);
+  }
+  if (lane < 16) {
+    double* xo = Xd + p * 16 * XDS;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) xo[k * XDS + c] = x[k];
+  }
+  if (lane == 0 && badmask) {
+    const int j = __ffs(badmask) - 1;
+    if (c0 + j < n)
+      atomicCAS(reinterpret_cast<unsigned long long*>(bad_pivot),
+                static_cast<unsigned long long>(-1ll),
+                static_cast<unsigned long long>(d - 1 - (gcol0 + c0 + j)));
+  }
+}
+
 __global__ void __launch_bounds__(LEAF_THREADS, 1)
-leaf_kernel(double* __restrict__ A, double* __restrict__ Mt, double* __restrict__ Xout, int d,
-            int off, int n, long long* __restrict__ bad_pivot) {
+leaf_kernel(const double* __restrict__ A, double* __restrict__ Mt, double* __restrict__ Xout,
+            int d, int off, int n, long long* __restrict__ bad_pivot) {
   extern __shared__ __align__(16) double lsm[];
-  const long long o = off;
-  leaf_factor_invert(A + o * d + o, d, n, Xout, Mt + o * d + o, d, bad_pivot, off, d, lsm);
+  double* S = lsm;
+  double* Xd = lsm + NB * LS;
+  const double* Ab = A + static_cast<long long>(off) * d + off;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t4 = lane & 3;
+
+  {  // rows r < n up to the end of their diagonal 16-block, in 16-byte chunks
+    for (int r = warp; r < n; r += LEAF_THREADS / 32) {
+      const int cend = min(n, 16 * (r / 16 + 1));
+      for (int c = 2 * lane; c < cend; c += 64)
+        cp_async16(smem_u32(S + r * LS + c), Ab + static_cast<long long>(r) * d + c, 16);
+    }
+    cp_async_commit();
+    // meanwhile zero the strictly-upper 16-blocks (R starts at 0 there) and
+    // make rows past n identity rows; 16-column segments, 8 per row
+    for (int sg = tid; sg < NB * 8; sg += LEAF_THREADS) {
+      const int r = sg >> 3, b = sg & 7;
+      if (r >= n || b > (r >> 4)) {
+        double2* z = reinterpret_cast<double2*>(S + r * LS + 16 * b);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) z[i] = make_double2(0.0, 0.0);
+        if (r >= n && b == (r >> 4)) S[r * LS + r] = 1.0;
+      }
+    }
+    cp_async_wait<0>();
+  }
+  __syncthreads();
+  if (warp == 0) leaf_diag_factor(S, Xd, 0, n, off, d, bad_pivot, lane);
+
+  // fragment element (r, c) of a 16 x 16 block, r = 8 rt + g, c = 8 ct + 2 t4 + e
+  auto frag_rc = [=](int rt, int ct, int e, int& r, int& c) {
+    r = 8 * rt + g;
+    c = 8 * ct + 2 * t4 + e;
+  };
+  for (int p = 0; p < 8; ++p) {
+    __syncthreads();  // X_pp is in Xd[p]; the previous panel's updates are done
+    const double* Xp = Xd + p * 16 * XDS;
+    if (warp < 7) {  // (ii): 7 - p blocks below, p blocks to the left
+      double acc[2][2][2] = {};
+      if (warp < 7 - p) {  // L_ip = A_ip X_pp^T, in place
+        double* blk = S + 16 * (p + 1 + warp) * LS + 16 * p;
+        blk16_mma(acc, [=](int r, int q) { return blk[r * LS + q]; },
+                  [=](int q, int c) { return Xp[c * XDS + q]; }, lane);
+#pragma unroll
+        for (int rt = 0; rt < 2; ++rt)
+#pragma unroll
+          for (int ct = 0; ct < 2; ++ct)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              int r, c;
+              frag_rc(rt, ct, e, r, c);
+              blk[r * LS + c] = acc[rt][ct][e];
+            }
+      } else {  // X_pj = X_pp R_pj; R_pj^T sits at block (j, p)
+        double* bt = S + 16 * (warp - (7 - p)) * LS + 16 * p;   // R_pj(q, c) = bt[c * LS + q]
+        blk16_mma(acc, [=](int r, int q) { return Xp[r * XDS + q]; },
+                  [=](int q, int c) { return bt[c * LS + q]; }, lane);
+#pragma unroll
+        for (int rt = 0; rt < 2; ++rt)
+#pragma unroll
+          for (int ct = 0; ct < 2; ++ct)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              int r, c;
+              frag_rc(rt, ct, e, r, c);
+              bt[c * LS + r] = acc[rt][ct][e];
+            }
+        // X_pj is final: its rows of Xout (row-major X), two columns per store
+        const int j = warp - (7 - p);
+#pragma unroll
+        for (int rt = 0; rt < 2; ++rt)
+#pragma unroll
+          for (int ct = 0; ct < 2; ++ct) {
+            int r, c;
+            frag_rc(rt, ct, 0, r, c);
+            *reinterpret_cast<double2*>(Xout + (16 * p + r) * NB + 16 * j + c) =
+                make_double2(acc[rt][ct][0], acc[rt][ct][1]);
+          }
+      }
+    }
+    __syncthreads();  // L_ip and X_pj are complete
+    if (p == 7) break;
+    // (iii): A_ik -= L_ip L_kp^T (p < k <= i) and R_ij -= L_ip X_pj (i > p, j <= p)
+    auto job_a = [&](int i, int k) {
+      double* C = S + 16 * i * LS + 16 * k;
+      const double* Li = S + 16 * i * LS + 16 * p;
+      const double* Lk = S + 16 * k * LS + 16 * p;
+      double acc[2][2][2];
+#pragma unroll
+      for (int rt = 0; rt < 2; ++rt)
+#pragma unroll
+        for (int ct = 0; ct < 2; ++ct)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            int r, c;
+            frag_rc(rt, ct, e, r, c);
+            acc[rt][ct][e] = C[r * LS + c];
+          }
+      blk16_mma(acc, [=](int r, int q) { return Li[r * LS + q]; },
+                [=](int q, int c) { return -Lk[c * LS + q]; }, lane);
+#pragma unroll
+      for (int rt = 0; rt < 2; ++rt)
+#pragma unroll
+        for (int ct = 0; ct < 2; ++ct)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            int r, c;
+            frag_rc(rt, ct, e, r, c);
+            C[r * LS + c] = acc[rt][ct][e];
+          }
+    };
+    auto job_r = [&](int i, int j) {
+      double* RT = S + 16 * j * LS + 16 * i;        // R_ij(r, c) = RT[c * LS + r]
+      const double* Li = S + 16 * i * LS + 16 * p;
+      const double* XT = S + 16 * j * LS + 16 * p;  // X_pj(q, c) = XT[c * LS + q], j < p
+      double acc[2][2][2];
+#pragma unroll
+      for (int rt = 0; rt < 2; ++rt)
+#pragma unroll
+        for (int ct = 0; ct < 2; ++ct)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            int r, c;
+            frag_rc(rt, ct, e, r, c);
+            acc[rt][ct][e] = RT[c * LS + r];
+          }
+      if (j < p)
+        blk16_mma(acc, [=](int r, int q) { return Li[r * LS + q]; },
+                  [=](int q, int c) { return -XT[c * LS + q]; }, lane);
+      else
+        blk16_mma(acc, [=](int r, int q) { return Li[r * LS + q]; },
+                  [=](int q, int c) { return -Xp[q * XDS + c]; }, lane);
+#pragma unroll
+      for (int rt = 0; rt < 2; ++rt)
+#pragma unroll
+        for (int ct = 0; ct < 2; ++ct)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            int r, c;
+            frag_rc(rt, ct, e, r, c);
+            RT[c * LS + r] = acc[rt][ct][e];
+          }
+    };
+    if (warp == 0) {  // the next diagonal block first, then its factorization
+      job_a(p + 1, p + 1);
+      __syncwarp();
+      leaf_diag_factor(S, Xd, p + 1, n, off, d, bad_pivot, lane);
+    } else {
+      const int na = (7 - p) * (8 - p) / 2, nr = (7 - p) * (p + 1);
+      for (int jb = warp - 1; jb < na - 1 + nr; jb += 7) {
+        if (jb < na - 1) {
+          int a = jb + 1, k = p + 1;  // pairs (i, k), k = p+1..7, i = k..7; pair 0 is warp 0's
+          while (a >= 8 - k) { a -= 8 - k; ++k; }
+          job_a(k + a, k);
+        } else {
+          const int r = jb - (na - 1);
+          job_r(p + 1 + r / (p + 1), r % (p + 1));
+        }
+      }
+    }
+  }
+  __syncthreads();
+  // Xout: the diagonal blocks from Xd and zeros above them (the blocks
+  // below were written as they were formed); consecutive lanes take
+  // consecutive 16-byte pieces of a row
+  double2* Xo2 = reinterpret_cast<double2*>(Xout);
+  for (int i2 = tid; i2 < NB * NB / 2; i2 += LEAF_THREADS) {
+    const int r = i2 >> 6, c = (i2 & 63) * 2;
+    const int br = r >> 4, bc = c >> 4;
+    if (bc > br)
+      Xo2[i2] = make_double2(0.0, 0.0);
+    else if (bc == br)
+      Xo2[i2] = *reinterpret_cast<const double2*>(Xd + br * 16 * XDS + (r & 15) * XDS + (c & 15));
+  }
+  // X^T into the n x n block of Mt: S's strict upper blocks hold it; the
+  // diagonal blocks are X_pp^T; zero below the diagonal
+  double* Mb = Mt + static_cast<long long>(off) * d + off;
+  for (int r = warp; r < n; r += LEAF_THREADS / 32) {
+    const int br = r >> 4;
+    for (int c = 2 * lane; c < n; c += 64) {
+      double v0, v1;
+      const int bc = c >> 4;
+      if (bc > br) {
+        const double2 v = *reinterpret_cast<const double2*>(S + r * LS + c);
+        v0 = v.x;
+        v1 = v.y;
+      } else if (bc == br) {
+        const double* xd = Xd + br * 16 * XDS;
+        const int a = r & 15, b0 = c & 15;
+        v0 = (b0 >= a) ? xd[b0 * XDS + a] : 0.0;
+        v1 = (b0 + 1 >= a) ? xd[(b0 + 1) * XDS + a] : 0.0;
+      } else {
+        v0 = v1 = 0.0;
+      }
+      *reinterpret_cast<double2*>(Mb + static_cast<long long>(r) * d + c) = make_double2(v0, v1);
+    }
+  }
 }
 
 // ------------------------------------------------------------ NT DGEMM
 // C[m][n] = alpha * sum_k A[m][k] B[n][k] + beta * C[m][n]  for up to MAXP
-// problems per launch.  TM x 128 tile per CTA, 8 warps in a WGM x (8/WGM)
+// problems per launch.  TM x 128 tile per CTA, NW warps in a WGM x (NW/WGM)
 // grid, each warp an (MI*8) x (NI*8) block of m8n8k4 fp64 MMAs.  A and B
 // slices of 16 along K are copied by cp.async (16-byte chunks, zero fill
 // outside the matrix) into [row][k] tiles padded to 20 doubles per row, so
 // both the copies and the fragment reads are free of bank conflicts.
 constexpr int TN = 128, TK = 16, LDS = TK + 4, GSTAGES = 3;
-constexpr int GEMM_THREADS = 256;
 constexpr int MAXP = 64;
 
 struct GemmProblem {
@@ -369,14 +448,15 @@ template <int TM>
 constexpr int gemm_smem() {
   return GSTAGES * (TM + TN) * LDS * 8;
 }
-constexpr int LEAF_SMEM = (4 * NB + 32 + NB * TS + NB * 4) * 8;
 
 
 
-template <int TM, int WGM>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
+// NW warps (NW * 32 threads) in a WGM x (NW / WGM) grid.
+template <int TM, int WGM, int NW = 8>
+__global__ void __launch_bounds__(NW * 32, 1)
 dgemm_nt_kernel(const __grid_constant__ GemmBatch batch) {
-  constexpr int WGN = 8 / WGM;
+  constexpr int NTHREADS = NW * 32;
+  constexpr int WGN = NW / WGM;
   constexpr int WM = TM / WGM, WN = TN / WGN;
   constexpr int MI = WM / 8, NI = WN / 8;
   extern __shared__ __align__(16) double gsm[];
@@ -418,7 +498,7 @@ dgemm_nt_kernel(const __grid_constant__ GemmBatch batch) {
     const int k0 = slice * TK;
     const uint32_t sa = smem_u32(As + stage * TM * LDS);
     const uint32_t sb = smem_u32(Bs + stage * TN * LDS);
-    for (int c = tid; c < (TM + TN) * (TK / 2); c += GEMM_THREADS) {
+    for (int c = tid; c < (TM + TN) * (TK / 2); c += NTHREADS) {
       const bool isA = c < TM * (TK / 2);
       const int cc = isA ? c : c - TM * (TK / 2);
       const int row = cc >> 3, kc = (cc & 7) * 2;
@@ -440,7 +520,7 @@ dgemm_nt_kernel(const __grid_constant__ GemmBatch batch) {
     }
     const GemmProblem& q = *T.q;
     if (q.beta != 0.0) {  // pull this tile of C into L2 for the epilogue
-      for (int c = tid; c < TM * 8; c += GEMM_THREADS) {
+      for (int c = tid; c < TM * 8; c += NTHREADS) {
         const int row = c >> 3, col = T.n0 + (c & 7) * 16;
         if (T.m0 + row < q.M && col < q.N)
           asm volatile("prefetch.global.L2 [%0];" ::"l"(q.C + static_cast<long long>(T.m0 + row) * q.ldc + col));
@@ -466,17 +546,26 @@ dgemm_nt_kernel(const __grid_constant__ GemmBatch batch) {
       const int stg = (g + sl) % GSTAGES;
       const double* a_s = As + stg * TM * LDS + (wm * WM + (lane >> 2)) * LDS + (lane & 3);
       const double* b_s = Bs + stg * TN * LDS + (wn * WN + (lane >> 2)) * LDS + (lane & 3);
+      // fragments double-buffered: step kk+1's loads are in flight while
+      // step kk's MMAs issue
+      double af[2][MI], bf[2][NI];
+#pragma unroll
+      for (int i = 0; i < MI; ++i) af[0][i] = a_s[i * 8 * LDS];
+#pragma unroll
+      for (int j = 0; j < NI; ++j) bf[0][j] = b_s[j * 8 * LDS];
 #pragma unroll
       for (int kk = 0; kk < TK / 4; ++kk) {
-        double af[MI], bf[NI];
+        const int cb = kk & 1;
+        if (kk + 1 < TK / 4) {
 #pragma unroll
-        for (int i = 0; i < MI; ++i) af[i] = a_s[i * 8 * LDS + kk * 4];
+          for (int i = 0; i < MI; ++i) af[cb ^ 1][i] = a_s[i * 8 * LDS + (kk + 1) * 4];
 #pragma unroll
-        for (int j = 0; j < NI; ++j) bf[j] = b_s[j * 8 * LDS + kk * 4];
+          for (int j = 0; j < NI; ++j) bf[cb ^ 1][j] = b_s[j * 8 * LDS + (kk + 1) * 4];
+        }
 #pragma unroll
         for (int i = 0; i < MI; ++i)
 #pragma unroll
-          for (int j = 0; j < NI; ++j) dmma_8x8x4(acc[i][j][0], acc[i][j][1], af[i], bf[j]);
+          for (int j = 0; j < NI; ++j) dmma_8x8x4(acc[i][j][0], acc[i][j][1], af[cb][i], bf[cb][j]);
       }
     }
     g += cur.ns;

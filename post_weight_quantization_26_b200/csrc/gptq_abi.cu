@@ -89,6 +89,9 @@ gptq_status device_setup(int* num_sms) {
     GPTQ_CUDA_TRY(cudaFuncSetAttribute(syrk::syrk_bf16_tcgen05_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        syrk::SMEM_BYTES));
+    GPTQ_CUDA_TRY(cudaFuncSetAttribute(chol::dgemm_nt_kernel<128, 4, 16>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       chol::gemm_smem<128>()));
     GPTQ_CUDA_TRY(cudaFuncSetAttribute(chol::dgemm_nt_kernel<128, 2>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        chol::gemm_smem<128>()));
@@ -241,7 +244,7 @@ namespace {
 // it (a persistent grid on every SM would keep a later kernel on another
 // stream from starting until it exits).  Problems with an empty output are
 // dropped.
-template <int TM, int WGM>
+template <int TM, int WGM, int NW = 8>
 gptq_status launch_nt(const std::vector<chol::GemmProblem>& probs, cudaStream_t s,
                       int reserve_sms = 0) {
   int num_sms = 148;
@@ -262,7 +265,7 @@ gptq_status launch_nt(const std::vector<chol::GemmProblem>& probs, cudaStream_t 
     b.tile_start[b.count] = tiles;
     const int grid = std::min(tiles, std::max(1, num_sms - reserve_sms));
     if (grid > 0) {
-      chol::dgemm_nt_kernel<TM, WGM><<<grid, chol::GEMM_THREADS, chol::gemm_smem<TM>(), s>>>(b);
+      chol::dgemm_nt_kernel<TM, WGM, NW><<<grid, NW * 32, chol::gemm_smem<TM>(), s>>>(b);
       GPTQ_LAUNCH_CHECK();
     }
   }
@@ -472,7 +475,7 @@ gptq_status gptq_prepare_hinv(const float* H, int64_t d, double damp_rel, float*
     }
     // two SMs stay free for D_k and leaf k+1 on the auxiliary stream (the
     // leaf's 141 KB of shared memory cannot share an SM with a U_k CTA)
-    st = launch_nt<128, 2>(uk, s, 2);
+    st = launch_nt<128, 4, 16>(uk, s, 2);
     if (st != GPTQ_OK) return st;
     GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, evL[k & 1], 0));  // X_{k+1} for P_{k+1}
   }
