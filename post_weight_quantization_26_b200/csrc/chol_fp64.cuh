@@ -471,9 +471,18 @@ dgemm_nt_kernel(const __grid_constant__ GemmBatch batch) {
   int t = bid;
   const int step = static_cast<int>(gridDim.x);
 
-  struct Tile { const GemmProblem* q; int m0, n0, ns; };
+  // A tile's problem lives in registers (the batch is only read here, once
+  // per tile: fields read through a pointer into the parameter block would
+  // be reloaded from memory at every use).
+  struct Tile {
+    const double* A;
+    const double* B;
+    double* C;
+    long long lda, ldb, ldc;
+    int M, N, K, m0, n0, ns;
+    double alpha, beta;
+  };
   auto decode = [&](int tt) {
-    Tile T;
     int pi = 0;
     while (pi + 1 < batch.count && batch.tile_start[pi + 1] <= tt) ++pi;
     const GemmProblem& q = batch.p[pi];
@@ -490,26 +499,40 @@ dgemm_nt_kernel(const __grid_constant__ GemmBatch batch) {
       tm_i = lt / tn;
       tn_i = lt - tm_i * tn;
     }
-    T.q = &q; T.m0 = tm_i * TM; T.n0 = tn_i * TN; T.ns = (q.K + TK - 1) / TK;
+    Tile T;
+    T.A = q.A; T.B = q.B; T.C = q.C;
+    T.lda = q.lda; T.ldb = q.ldb; T.ldc = q.ldc;
+    T.M = q.M; T.N = q.N; T.K = q.K;
+    T.alpha = q.alpha; T.beta = q.beta;
+    T.m0 = tm_i * TM; T.n0 = tn_i * TN; T.ns = (q.K + TK - 1) / TK;
     return T;
   };
+  // Each thread copies APT 16-byte pieces of A and CPT - APT of B per slice,
+  // all in the same k column, RSTEP rows apart.
+  constexpr int CPT = (TM + TN) * (TK / 2) / NTHREADS;
+  constexpr int APT = TM * (TK / 2) / NTHREADS;
+  constexpr int RSTEP = NTHREADS / (TK / 2);
+  static_assert(CPT * NTHREADS == (TM + TN) * (TK / 2) && APT * NTHREADS == TM * (TK / 2),
+                "the copies must split evenly over the threads");
+  const int crow0 = tid / (TK / 2), ckc = (tid % (TK / 2)) * 2;
   auto issue = [&](const Tile& T, int slice, int stage) {
-    const GemmProblem& q = *T.q;
-    const int k0 = slice * TK;
-    const uint32_t sa = smem_u32(As + stage * TM * LDS);
-    const uint32_t sb = smem_u32(Bs + stage * TN * LDS);
-    for (int c = tid; c < (TM + TN) * (TK / 2); c += NTHREADS) {
-      const bool isA = c < TM * (TK / 2);
-      const int cc = isA ? c : c - TM * (TK / 2);
-      const int row = cc >> 3, kc = (cc & 7) * 2;
-      const int grow = (isA ? T.m0 : T.n0) + row;
-      const int lim = isA ? q.M : q.N;
-      const double* base = isA ? q.A : q.B;
-      const long long ld = isA ? q.lda : q.ldb;
-      const bool ok = grow < lim && k0 + kc < q.K;
-      const double* src = ok ? base + static_cast<long long>(grow) * ld + k0 + kc : base;
-      const uint32_t dst = (isA ? sa : sb) + (row * LDS + kc) * 8;
-      cp_async16(dst, src, ok ? 16 : 0);
+    const int k = slice * TK + ckc;
+    const bool kin = k < T.K;
+    const uint32_t sa = smem_u32(As + stage * TM * LDS) + (crow0 * LDS + ckc) * 8;
+    const uint32_t sb = smem_u32(Bs + stage * TN * LDS) + (crow0 * LDS + ckc) * 8;
+#pragma unroll
+    for (int i = 0; i < APT; ++i) {
+      const int grow = T.m0 + crow0 + i * RSTEP;
+      const bool ok = kin && grow < T.M;
+      const double* src = ok ? T.A + static_cast<long long>(grow) * T.lda + k : T.A;
+      cp_async16(sa + i * RSTEP * LDS * 8, src, ok ? 16 : 0);
+    }
+#pragma unroll
+    for (int i = 0; i < CPT - APT; ++i) {
+      const int grow = T.n0 + crow0 + i * RSTEP;
+      const bool ok = kin && grow < T.N;
+      const double* src = ok ? T.B + static_cast<long long>(grow) * T.ldb + k : T.B;
+      cp_async16(sb + i * RSTEP * LDS * 8, src, ok ? 16 : 0);
     }
   };
   auto prologue = [&](const Tile& T, int g0) {
@@ -518,12 +541,11 @@ dgemm_nt_kernel(const __grid_constant__ GemmBatch batch) {
       if (st < T.ns) issue(T, st, (g0 + st) % GSTAGES);
       cp_async_commit();
     }
-    const GemmProblem& q = *T.q;
-    if (q.beta != 0.0) {  // pull this tile of C into L2 for the epilogue
+    if (T.beta != 0.0) {  // pull this tile of C into L2 for the epilogue
       for (int c = tid; c < TM * 8; c += NTHREADS) {
         const int row = c >> 3, col = T.n0 + (c & 7) * 16;
-        if (T.m0 + row < q.M && col < q.N)
-          asm volatile("prefetch.global.L2 [%0];" ::"l"(q.C + static_cast<long long>(T.m0 + row) * q.ldc + col));
+        if (T.m0 + row < T.M && col < T.N)
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(T.C + static_cast<long long>(T.m0 + row) * T.ldc + col));
       }
     }
   };
@@ -532,7 +554,7 @@ dgemm_nt_kernel(const __grid_constant__ GemmBatch batch) {
   Tile cur;
   if (t < total) { cur = decode(t); prologue(cur, g); }
   while (t < total) {
-    const GemmProblem& q = *cur.q;
+    const Tile& q = cur;
     double acc[MI][NI][2];
 #pragma unroll
     for (int i = 0; i < MI; ++i)
