@@ -115,6 +115,26 @@ struct StepSmem {
 template <int B>
 constexpr int block_step_smem() { return StepSmem<B>::BYTES; }
 
+// x = hi + lo with hi a TF32 value (low 13 mantissa bits cleared); both
+// returned as the bit patterns the tf32 MMA reads.
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+  hi = __float_as_uint(x) & 0xFFFFE000u;
+  lo = __float_as_uint(x - __uint_as_float(hi));
+}
+
+// D += A B, m16n8k8, A row-major tf32 (a0: row g col t, a1: row g+8 col t,
+// a2: row g col t+4, a3: row g+8 col t+4; g = lane/4, t = lane%4), B
+// column-major (b0: row t col g, b1: row t+4 col g), fp32 accumulators
+// (d0, d1: row g cols 2t, 2t+1; d2, d3: row g+8).
+__device__ __forceinline__ void mma_tf32_m16n8k8(float (&d)[4], const uint32_t (&a)[4],
+                                                 uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 template <int B>
 __device__ __forceinline__ void stage_rows(float* dst, const float* src, long long ld, int r0,
                                            int d_row, int ncols, int tid) {
@@ -195,31 +215,63 @@ block_step_kernel(const float* __restrict__ Wk, int d_row, int d_col, int j0, in
   float* wrow = Ws + rloc * LDG;
   float* erow = Es + rloc * LDG;
   if (jp0 >= 0) {
-    // (a) W[rows, blk] -= E_prev[rows] * G[prev blk, blk]  (thread t: chunks t, t+4, ...)
-    constexpr int NCH = B / 16;
-    float4 w4[NCH];
+    // (a) W[rows, blk] -= E_prev[rows] * G[prev blk, blk] on the MMA path:
+    // m16n8k8 tf32, three products of the split operands (hi hi + hi lo +
+    // lo hi; hi = the low 13 mantissa bits cleared), fp32 accumulate, the
+    // same arithmetic as the trailing update.  Warp w takes the output
+    // columns [w B/4, (w+1) B/4) of both 16-row halves of the slab; ncols is
+    // a multiple of 32, so a warp's columns are all inside or all past it.
+    {
+      constexpr int NTW = B / 32;  // 8-column tiles per warp
+      const int warp = tid >> 5, g = lane >> 2, t4 = lane & 3;
+      const int cw = warp * (B / 4);
+      if (cw < ncols) {
+        float acc[2][NTW][4];
 #pragma unroll
-    for (int i = 0; i < NCH; ++i) {
-      const int col = 16 * i + 4 * t;
-      w4[i] = (col < ncols) ? *reinterpret_cast<const float4*>(wrow + col)
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-#pragma unroll 4
-    for (int p = 0; p < B; ++p) {
-      const float e = erow[p];
-      const float* gr = Gs + p * LDG + 4 * t;
+        for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-      for (int i = 0; i < NCH; ++i) {
-        if (16 * i + 4 * t >= ncols) continue;
-        const float4 g4 = *reinterpret_cast<const float4*>(gr + 16 * i);
-        w4[i].x = fmaf(-e, g4.x, w4[i].x); w4[i].y = fmaf(-e, g4.y, w4[i].y);
-        w4[i].z = fmaf(-e, g4.z, w4[i].z); w4[i].w = fmaf(-e, g4.w, w4[i].w);
+          for (int nt = 0; nt < NTW; ++nt) {
+            const float* w0 = Ws + (16 * mt + g) * LDG + cw + 8 * nt + 2 * t4;
+            acc[mt][nt][0] = w0[0];
+            acc[mt][nt][1] = w0[1];
+            acc[mt][nt][2] = w0[8 * LDG];
+            acc[mt][nt][3] = w0[8 * LDG + 1];
+          }
+#pragma unroll 2
+        for (int k0 = 0; k0 < B; k0 += 8) {
+          uint32_t ah[2][4], al[2][4];
+#pragma unroll
+          for (int mt = 0; mt < 2; ++mt) {
+            const float* e0 = Es + (16 * mt + g) * LDG + k0 + t4;
+            const float v[4] = {-e0[0], -e0[8 * LDG], -e0[4], -e0[8 * LDG + 4]};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) split_tf32(v[q], ah[mt][q], al[mt][q]);
+          }
+#pragma unroll
+          for (int nt = 0; nt < NTW; ++nt) {
+            const float* g0 = Gs + (k0 + t4) * LDG + cw + 8 * nt + g;
+            uint32_t bh0, bl0, bh1, bl1;
+            split_tf32(g0[0], bh0, bl0);
+            split_tf32(g0[4 * LDG], bh1, bl1);
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt) {
+              mma_tf32_m16n8k8(acc[mt][nt], ah[mt], bh0, bh1);
+              mma_tf32_m16n8k8(acc[mt][nt], ah[mt], bl0, bl1);
+              mma_tf32_m16n8k8(acc[mt][nt], al[mt], bh0, bh1);
+            }
+          }
+        }
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+          for (int nt = 0; nt < NTW; ++nt) {
+            float* w0 = Ws + (16 * mt + g) * LDG + cw + 8 * nt + 2 * t4;
+            w0[0] = acc[mt][nt][0];
+            w0[1] = acc[mt][nt][1];
+            w0[8 * LDG] = acc[mt][nt][2];
+            w0[8 * LDG + 1] = acc[mt][nt][3];
+          }
       }
-    }
-#pragma unroll
-    for (int i = 0; i < NCH; ++i) {
-      const int col = 16 * i + 4 * t;
-      if (col < ncols) *reinterpret_cast<float4*>(wrow + col) = w4[i];
     }
     __syncthreads();  // every thread is done with the previous block's G rows
     stage_gblock<B>(Gs, G, d_col, j0, j0, ncols, ncols, tid);
