@@ -3,18 +3,20 @@
 // factor of H^-1), blocks of B columns with immediate in-block updates and
 // one lazy batched update of the columns to the right after each block.
 //
-// Per block j0:
-//   block_quant_kernel   the B columns of every row: parameters at a group
-//                        start, code, dequantize, e = (w - w^)/G_qq, subtract
-//                        e * G[q, k] from the later columns of the block,
-//                        keep e in E; then bit-pack the block's codes.
-//                        A row's B values live in registers of 4 threads
-//                        (interleaved in 4-column chunks); G's diagonal
-//                        block sits in shared memory and is read as
-//                        broadcast float4s; e crosses the 4 threads by shuffle.
-//   trailing_update_kernel  W[:, j0+B:] -= E * G[j0:j0+B, j0+B:]  (fp32 FFMA,
-//                        128x128 register-tiled).
-//
+// Per block j0 (block_step_kernel, one CTA per 32 rows):
+//   (a) apply the previous block's errors to this block, W -= E_prev G
+//       (m16n8k8 tf32 MMAs on the split operands);
+//   (b) the B columns of every row: parameters at a group start, code,
+//       dequantize, e = (w - w^)/G_qq, subtract e * G[q, k] from the later
+//       columns of the block, keep e in E.  A row's values live in
+//       registers of 4 threads (interleaved in 4-column chunks); G's
+//       diagonal block sits in shared memory and is read as broadcast
+//       float4s; e crosses the 4 threads by shuffle;
+//   (c) write E as a TF32 split for the trailing update and bit-pack the
+//       block's codes.
+// The columns right of block j0 + B are updated by trailing_tf32x3_kernel
+// (trailing_tf32.cuh).
+
 // Quantizer (dingiv.github.io page, section 量化基础; youleyou.com page,
 // sections 二 and 四): asymmetric q = clip(rint(w/s) + z, 0, 2^b-1) with
 // s = (max(0,max) - min(0,min)) / (2^b-1), z = rint(-min(0,min)/s);
@@ -109,7 +111,8 @@ struct StepSmem {
   static constexpr int E_OFF = W_OFF + QROWS * LDG * 4;
   static constexpr int INV_OFF = E_OFF + QROWS * LDG * 4;
   static constexpr int C_OFF = INV_OFF + B * 4;
-  static constexpr int BYTES = C_OFF + QROWS * B;
+  static constexpr int LDC = B + 4;  // code row stride (bytes): the 8 rows of a warp on 8 banks
+  static constexpr int BYTES = C_OFF + QROWS * LDC;
 };
 
 template <int B>
@@ -333,7 +336,7 @@ block_step_kernel(const float* __restrict__ Wk, int d_row, int d_col, int j0, in
         qf = fminf(fmaxf(qf, 0.0f), maxq);
         const float xh = s * (qf - z);
         e = (x - xh) * invd[q];
-        codes[rloc * B + q] = static_cast<uint8_t>(qf);
+        codes[rloc * L::LDC + q] = static_cast<uint8_t>(qf);
         erow[q] = e;
       }
       e = __shfl_sync(0xffffffffu, e, qbase | tq);
@@ -388,7 +391,7 @@ block_step_kernel(const float* __restrict__ Wk, int d_row, int d_col, int j0, in
     const int nw = ncols * bits / 32;
     const size_t row_words = static_cast<size_t>(d_col) * bits / 32;
     uint32_t* qrow = qweight + static_cast<size_t>(r) * row_words + (static_cast<size_t>(j0) * bits) / 32;
-    const uint8_t* cs = codes + rloc * B;
+    const uint8_t* cs = codes + rloc * L::LDC;
     for (int wi = t; wi < nw; wi += 4) {
       const int bit0 = 32 * wi;
       const int kf = bit0 / bits, kl = (bit0 + 31) / bits;
@@ -399,90 +402,6 @@ block_step_kernel(const float* __restrict__ Wk, int d_row, int d_col, int j0, in
         val |= (sh >= 0) ? (c << sh) : (c >> (-sh));
       }
       qrow[wi] = val;
-    }
-  }
-}
-
-// W[:, n0:] -= E * G[j0:j0+K, n0:]  -- C (ldc = d_col) -= A (ld K) * B (ld d_col).
-constexpr int UT = 128, UK = 16, UTHREADS = 256;
-
-__global__ void __launch_bounds__(UTHREADS, 1)
-trailing_update_kernel(float* __restrict__ C, const float* __restrict__ A,
-                       const float* __restrict__ Bm, int M, int N, int K, int ldc, int ldb) {
-  __shared__ __align__(16) float As[2][UK][UT];
-  __shared__ __align__(16) float Bs[2][UK][UT];
-  const int m0 = blockIdx.x * UT, n0 = blockIdx.y * UT;
-  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-  float acc[8][8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
-
-  float4 ra[2], rb[2];
-  auto load = [&](int k0) {
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int idx = tid + e * UTHREADS;  // 512 float4 per operand slice
-      const int am = idx >> 2, ak = (idx & 3) * 4;  // A: 128 rows x 16 k
-      ra[e] = (m0 + am < M) ? *reinterpret_cast<const float4*>(A + static_cast<size_t>(m0 + am) * K + k0 + ak)
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
-      const int bk = idx >> 5, bn = (idx & 31) * 4;  // B: 16 k x 128 cols
-      rb[e] = (n0 + bn < N) ? *reinterpret_cast<const float4*>(Bm + static_cast<size_t>(k0 + bk) * ldb + n0 + bn)
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-  };
-  auto store = [&](int buf) {
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int idx = tid + e * UTHREADS;
-      const int am = idx >> 2, ak = (idx & 3) * 4;
-      As[buf][ak][am] = ra[e].x; As[buf][ak + 1][am] = ra[e].y;
-      As[buf][ak + 2][am] = ra[e].z; As[buf][ak + 3][am] = ra[e].w;
-      const int bk = idx >> 5, bn = (idx & 31) * 4;
-      *reinterpret_cast<float4*>(&Bs[buf][bk][bn]) = rb[e];
-    }
-  };
-
-  load(0);
-  store(0);
-  __syncthreads();
-  int buf = 0;
-  for (int k0 = 0; k0 < K; k0 += UK) {
-    const bool more = k0 + UK < K;
-    if (more) load(k0 + UK);
-#pragma unroll
-    for (int k = 0; k < UK; ++k) {
-      const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][k][ty * 4]);
-      const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][k][64 + ty * 4]);
-      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[buf][k][tx * 4]);
-      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[buf][k][64 + tx * 4]);
-      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-      const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
-    }
-    if (more) {
-      store(buf ^ 1);
-      __syncthreads();
-      buf ^= 1;
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int gm = m0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + i - 4);
-    if (gm >= M) continue;
-    float* crow = C + static_cast<size_t>(gm) * ldc + n0;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int cn = h * 64 + tx * 4;
-      if (n0 + cn >= N) continue;  // N % 32 == 0, so a float4 is all in or all out
-      float4 c = *reinterpret_cast<float4*>(crow + cn);
-      c.x -= acc[i][4 * h]; c.y -= acc[i][4 * h + 1];
-      c.z -= acc[i][4 * h + 2]; c.w -= acc[i][4 * h + 3];
-      *reinterpret_cast<float4*>(crow + cn) = c;
     }
   }
 }
