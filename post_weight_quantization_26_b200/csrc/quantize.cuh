@@ -329,24 +329,27 @@ block_step_kernel(const float* __restrict__ Wk, int d_row, int d_col, int j0, in
     for (int u = 0; u < 16; ++u) {
       const int q = q0 + u;
       const int tq = u >> 2;
-      float e = 0.0f;
-      if (t == tq) {
-        const float x = w[u & 3];
-        float qf = rintf(x / s) + z;
-        qf = fminf(fmaxf(qf, 0.0f), maxq);
-        const float xh = s * (qf - z);
-        e = (x - xh) * invd[q];
+      // loads first (independent of this column's result), then the
+      // quantization on every lane, branch-free; the owner's result is kept
+      const float4 g4 = *reinterpret_cast<const float4*>(Gs + q * LDG + q0 + 4 * t);
+      const float iq = invd[q];
+      const bool own = (t == tq);
+      const float x = w[u & 3];
+      float qf = rintf(x / s) + z;
+      qf = fminf(fmaxf(qf, 0.0f), maxq);
+      const float xh = s * (qf - z);
+      const float eo = (x - xh) * iq;
+      if (own) {
         codes[rloc * L::LDC + q] = static_cast<uint8_t>(qf);
-        erow[q] = e;
+        erow[q] = eo;
       }
-      e = __shfl_sync(0xffffffffu, e, qbase | tq);
+      const float e = __shfl_sync(0xffffffffu, own ? eo : 0.0f, qbase | tq);
       if (u < 15) {
-        const float4 g4 = *reinterpret_cast<const float4*>(Gs + q * LDG + q0 + 4 * t);
         const int kb = 4 * t;
-        if (kb > u) w[0] = fmaf(-e, g4.x, w[0]);
-        if (kb + 1 > u) w[1] = fmaf(-e, g4.y, w[1]);
-        if (kb + 2 > u) w[2] = fmaf(-e, g4.z, w[2]);
-        if (kb + 3 > u) w[3] = fmaf(-e, g4.w, w[3]);
+        w[0] = (kb > u) ? fmaf(-e, g4.x, w[0]) : w[0];
+        w[1] = (kb + 1 > u) ? fmaf(-e, g4.y, w[1]) : w[1];
+        w[2] = (kb + 2 > u) ? fmaf(-e, g4.z, w[2]) : w[2];
+        w[3] = (kb + 3 > u) ? fmaf(-e, g4.w, w[3]) : w[3];
       }
     }
     __syncwarp();
