@@ -12,12 +12,13 @@
 // in the same sweep (block forward substitution on the identity) and kept
 // transposed (Mt = M^T, upper block triangle):
 //   leaf(k)  one CTA factors the diagonal block A_kk = L_kk L_kk^T and forms
-//            X_kk = L_kk^-1 in registers (column sweep, 4x4 tiles/thread);
+//            X_kk = L_kk^-1, in 16-column panels held in shared memory;
 //   P_k      L_ik = A_ik X_kk^T (rows below), Mt[:k, k] <- Mt[:k, k] X_kk^T;
-//   U_k      A_ij -= L_ik L_jk^T on the lower tiles (i, j > k) and
-//            Mt[:k+1, i] -= Mt[:k+1, k] L_ik^T for the rows i > k; the CTA
-//            that computes the next diagonal tile then runs leaf(k+1), so the
-//            serial leaf hides behind the rest of the update.
+//   D_k      the next diagonal block, A_{k+1,k+1} -= L_{k+1,k} L_{k+1,k}^T,
+//            then leaf(k+1), both on a second stream;
+//   U_k      A_ij -= L_ik L_jk^T on the other lower tiles (i, j > k) and
+//            Mt[:k+1, i] -= Mt[:k+1, k] L_ik^T for the rows i > k, on all
+//            SMs but two, so that D_k and the serial leaf run beside it.
 // Every product is an "NT" GEMM (both operands row-major along K) on the
 // fp64 MMA path (mma.sync m8n8k4 f64), staged by cp.async through a 3-deep
 // ring of padded shared-memory tiles.
