@@ -46,6 +46,9 @@ def parse_args():
     p.add_argument("--tokens", type=int, default=0,
                    help="calibration tokens (default: the workload's); a smaller "
                         "full-path configuration for profiling captures")
+    p.add_argument("--bits", type=int, default=0,
+                   help="code width (default: the workload's); same path, other clip/pack widths")
+    p.add_argument("--sym", action="store_true", help="symmetric quantizer instead of the workload's")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
@@ -171,6 +174,10 @@ def run_reference(args, rank, world):
         return
     from post_weight_quantization_26_b200 import synth
     spec = workload_spec(args.workload, 0)
+    if args.bits:
+        spec = spec.with_(bits=args.bits, name=f"{spec.name}_int{args.bits}")
+    if args.sym:
+        spec = spec.with_(sym=True, name=f"{spec.name}_sym")
     tokens = min(8192, spec.n_tokens)
     x_host = synth.gen_tokens(spec, 0, tokens)
     w_host = synth.gen_weight(spec)
@@ -259,6 +266,10 @@ def run_ours(args, rank, world, local_rank):
     spec = workload_spec(args.workload, rank)
     if args.tokens:
         spec = spec.with_(n_tokens=args.tokens, name=f"{spec.name}_n{args.tokens}")
+    if args.bits:
+        spec = spec.with_(bits=args.bits, name=f"{spec.name}_int{args.bits}")
+    if args.sym:
+        spec = spec.with_(sym=True, name=f"{spec.name}_sym")
     d, n, dr = spec.d_col, spec.n_tokens, spec.d_row
     cfg = G.make_config(bits=spec.bits, group_size=spec.group, sym=spec.sym,
                         block=spec.block, damp_rel=spec.damp)

@@ -48,7 +48,9 @@ typedef enum {
 } gptq_status;
 
 /* Quantizer settings.
- *  bits        2, 3 or 4.
+ *  bits        2 to 8 (the pages' INT2/3/4 outputs and INT8; every width
+ *              packs into the same little-endian bit stream, codes may
+ *              straddle 32-bit words).
  *  group_size  0 = one scale/zero per output channel, computed from the
  *              original row of W; otherwise the number of consecutive input
  *              columns sharing a scale/zero, computed from the current

@@ -134,7 +134,7 @@ gptq_status device_setup(int* num_sms) {
 
 bool config_ok(const gptq_config* c, int64_t d_col) {
   if (!c) return false;
-  if (c->bits < 2 || c->bits > 4) return false;
+  if (c->bits < 2 || c->bits > 8) return false;
   if (c->block != 32 && c->block != 64 && c->block != 128) return false;
   if (c->sym != 0 && c->sym != 1) return false;
   if (!(c->damp_rel >= 0.0) || !std::isfinite(c->damp_rel)) return false;

@@ -65,7 +65,7 @@ def test_workspace_size_rules(lib):
     # the fp64 factorization buffer dominates: d*d*8 bytes plus leaf inverses
     assert n >= 4096 * 4096 * 8
     assert n % 256 == 0
-    for bad in (G.make_config(bits=5), G.make_config(bits=1),
+    for bad in (G.make_config(bits=9), G.make_config(bits=1),
                 G.make_config(block=96), G.make_config(group_size=48),
                 G.make_config(group_size=96, block=128),
                 G.make_config(damp_rel=-1.0), G.GptqConfig(4, 0, 2, 128, 0.01)):
@@ -107,7 +107,7 @@ def test_prepare_and_quantize_validation(lib):
     q = lib.gptq_quantize_layer
     assert q(FAKE, 64, 100, FAKE, None, ctypes.byref(cfg), FAKE, FAKE, FAKE,
              FAKE, 1 << 30, None) == 1
-    bad = G.make_config(bits=7)
+    bad = G.make_config(bits=9)
     assert q(FAKE, 64, 128, FAKE, None, ctypes.byref(bad), FAKE, FAKE, FAKE,
              FAKE, 1 << 30, None) == 1
     assert q(FAKE, 64, 128, FAKE, None, ctypes.byref(cfg), FAKE, FAKE, FAKE,

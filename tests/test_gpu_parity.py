@@ -165,6 +165,10 @@ QCASES = [  # d_row, d_col, bits, group, sym, block
     (1, 32, 4, 0, False, 128),
     (130, 640, 4, 128, True, 128),
     (48, 256, 3, 64, False, 128),
+    (64, 384, 8, 0, False, 128),      # INT8, per channel
+    (96, 512, 8, 128, True, 128),     # INT8 symmetric, g = 128
+    (40, 320, 5, 32, False, 32),      # an odd width: codes straddle words
+    (64, 256, 6, 64, True, 64),
 ]
 
 
@@ -198,7 +202,25 @@ def test_quantize_matches_oracle(G, case):
         dtype=np.float32)
     _check_codes(codes, ref_codes)
     _check_codes(ze, ref_z)
-    np.testing.assert_allclose(sc, ref_s, rtol=1e-5)
+    _check_scales(sc, ref_s, codes, ref_codes, group, d_col)
+
+
+def _check_scales(sc, ref_s, codes, ref_codes, group, d_col):
+    """Scales within 1e-5 relative.  Group parameters are fitted to the
+    error-updated weights, so a permitted +-1 code difference earlier in a
+    row changes that row's later groups; those groups (and only those) are
+    held to a loose 1e-2.  Per-channel scales come from the original row and
+    are always held to 1e-5."""
+    sc, ref_s = np.asarray(sc, np.float64), np.asarray(ref_s, np.float64)
+    strict = np.ones(sc.shape, dtype=bool)
+    if group:
+        diff_cols = codes != ref_codes
+        first = np.where(diff_cols.any(1), diff_cols.argmax(1), d_col)
+        starts = np.arange(sc.shape[1]) * group
+        strict = starts[None, :] <= first[:, None]
+    rel = np.abs(sc - ref_s) / np.abs(ref_s)
+    assert rel[strict].max(initial=0) <= 1e-5, f"scale rel {rel[strict].max():.2e}"
+    assert rel.max(initial=0) <= 1e-2, f"scale rel {rel.max():.2e} after a code difference"
 
 
 def test_quantize_scaled_identity_is_rtn(G):
@@ -277,7 +299,8 @@ def test_end_to_end_small_256(G):
 
 
 @pytest.mark.parametrize("bits,group,sym", [(3, 128, False), (2, 0, True),
-                                            (4, 64, False)])
+                                            (4, 64, False), (8, 0, False),
+                                            (8, 128, True)])
 def test_end_to_end_variants(G, bits, group, sym):
     spec = synth.tiny_spec(192, 512, 3000, seed=bits * 7 + group).with_(
         bits=bits, group=group, sym=sym)
