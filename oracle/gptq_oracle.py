@@ -341,3 +341,23 @@ def unpack_codes(words, bits: int, cols: int) -> np.ndarray:
             v |= words[:, wi + 1] << np.uint64(32 - off)
         out[:, k] = (v & mask).astype(np.int64)
     return out
+
+
+# ---------------------------------------------------------------------------
+# Using the packed output: Y = X W^T with W dequantized (weight-only
+# quantized matmul; dingiv.github.io page, section GPTQ: the INT4 weights
+# serve inference, where memory-bound batch-1 decoding speeds up)
+# ---------------------------------------------------------------------------
+def dequantized_matmul(words, scales, zeros, x, bits: int, group: int) -> np.ndarray:
+    """``Y[b][r] = sum_k X[b][k] W^[r][k]`` in fp64, where ``W^`` is the
+    dequantized layer: ``W^[r][k] = s[r][g(k)] * (q[r][k] - z[r][g(k)])``
+    with ``q`` unpacked from ``words`` and ``g(k) = k // group`` (one group
+    per row when ``group`` is 0)."""
+    x = np.asarray(x, dtype=F64)
+    cols = x.shape[1]
+    q = unpack_codes(words, bits, cols).astype(F64)
+    s = np.asarray(scales, dtype=F64)
+    z = np.asarray(zeros, dtype=F64)
+    g = np.arange(cols) // (group if group else cols)
+    w_hat = s[:, g] * (q - z[:, g])
+    return x @ w_hat.T

@@ -331,3 +331,31 @@ def test_small_256_layer_end_to_end():
     assert ld < O.layer_loss_direct(w, O.rtn(w, 4)["w_hat"], x)
     r1 = O.gptq(w, h, bits=4, group=0, block=1, damp_rel=0.01)
     assert np.array_equal(r1["codes"], r["codes"])
+
+
+def test_dequantized_matmul_closed_forms():
+    """Codes equal to the zero point give Y = 0; unit scales, zero points 0
+    and all-ones codes give the row sums of X; a single code 3 at (r, k)
+    with scale 0.5 gives Y[:, r] = 1.5 X[:, k].  Grouped parameters pick
+    the right group (the second group's scale doubles its columns)."""
+    rng = np.random.default_rng(9)
+    bits, rows, cols = 4, 3, 64
+    x = rng.standard_normal((2, cols))
+    z = np.full((rows, 1), 5.0)
+    y0 = O.dequantized_matmul(O.pack_codes(np.full((rows, cols), 5), bits), np.ones((rows, 1)),
+                              z, x, bits, 0)
+    assert np.all(y0 == 0.0)
+    y1 = O.dequantized_matmul(O.pack_codes(np.ones((rows, cols), int), bits), np.ones((rows, 1)),
+                              np.zeros((rows, 1)), x, bits, 0)
+    np.testing.assert_allclose(y1, np.repeat(x.sum(1, keepdims=True), rows, 1), rtol=1e-12)
+    codes = np.zeros((rows, cols), int)
+    codes[1, 17] = 3
+    y2 = O.dequantized_matmul(O.pack_codes(codes, bits), np.full((rows, 1), 0.5),
+                              np.zeros((rows, 1)), x, bits, 0)
+    np.testing.assert_allclose(y2[:, 1], 1.5 * x[:, 17], rtol=1e-12)
+    assert np.all(y2[:, [0, 2]] == 0.0)
+    s = np.ones((rows, 2)); s[:, 1] = 2.0
+    y3 = O.dequantized_matmul(O.pack_codes(np.ones((rows, cols), int), bits), s,
+                              np.zeros((rows, 2)), x, bits, 32)
+    want = x[:, :32].sum(1) + 2.0 * x[:, 32:].sum(1)
+    np.testing.assert_allclose(y3, np.repeat(want[:, None], rows, 1), rtol=1e-12)
