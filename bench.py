@@ -49,6 +49,11 @@ def parse_args():
     p.add_argument("--bits", type=int, default=0,
                    help="code width (default: the workload's); same path, other clip/pack widths")
     p.add_argument("--sym", action="store_true", help="symmetric quantizer instead of the workload's")
+    p.add_argument("--w4a16", type=int, default=0, metavar="BATCH",
+                   help="instead of quantization, time the dequant-fused matmul of "
+                        "4-bit LLaMA-65B MLP layers with BATCH activation rows (1..8)")
+    p.add_argument("--w4a16-group", type=int, default=128, metavar="G",
+                   help="group size of the --w4a16 layers (0: one scale per output channel)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
@@ -460,6 +465,142 @@ def run_e2e(args, G, spec, cfg, x_host, w_host, dev, stream, world):
     return {"value": weak_value(world, dr, d, ms), "unit": UNIT, "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
+# ------------------------------------------------- dequant-fused matmul
+W4_METRIC = "W4A16 dequant-fused matmul, bytes streamed/s"
+W4_LAYERS = (("gate_proj", 22016, 8192), ("up_proj", 22016, 8192), ("down_proj", 8192, 22016))
+
+
+def run_w4a16(args, rank, world, local_rank):
+    """One step = the three 4-bit (g = 128 by default) LLaMA-65B MLP matmuls for one
+    batch of activation rows.  The packed layers total 271 MB, more than L2,
+    and run back to back, so every step streams them from HBM.  Each rank
+    runs its own copy (weak scaling, no collective)."""
+    import torch
+    import torch.distributed as dist
+
+    from post_weight_quantization_26_b200 import build as _build
+    from post_weight_quantization_26_b200 import gptq as G
+    from post_weight_quantization_26_b200 import synth
+
+    batch = args.w4a16
+    if rank == 0:
+        _build.build()
+    if world > 1:
+        dist.barrier()
+    G.load_library()
+    dev = torch.device("cuda", local_rank)
+    group = args.w4a16_group
+    cfg = G.make_config(bits=4, group_size=group)
+    layers, host = [], []
+    for i, (name, dr, dc) in enumerate(W4_LAYERS):
+        words, scales, zeros = synth.gen_packed_layer(dr, dc, group, seed=100 * rank + i)
+        xh = synth.gen_activations(batch, dc, seed=100 * rank + i).pin_memory()
+        layers.append((words.to(dev), scales.to(dev), zeros.to(dev), xh.to(dev),
+                       torch.empty((batch, dr), dtype=torch.float32, device=dev)))
+        host.append((xh, torch.empty((batch, dr), dtype=torch.float32).pin_memory()))
+    # algorithmic bytes: packed words + scales + zeros + X + Y, once per layer
+    layer_bytes = [dr * dc // 2 + dr * (dc // group if group else 1) * 5 + batch * dc * 2 + batch * dr * 4
+                   for _, dr, dc in W4_LAYERS]
+    step_bytes = sum(layer_bytes)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        for i, (wq, sc, ze, x, y) in enumerate(layers):
+            if ev:
+                ev[i][0].record(stream)
+            G.gptq_w4a16_matmul(wq, sc, ze, cfg, x, Y=y)
+            if ev:
+                ev[i][1].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    steps = max(1, args.steps)
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in W4_LAYERS]
+           for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    launches0 = G.gptq_launch_count()
+    t0.record(stream)
+    for i in range(steps):
+        step(evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    launches = G.gptq_launch_count() - launches0
+    clk = clocks.stop()
+    ms = max_over_ranks(t0.elapsed_time(t1) / steps, world, dev)
+    per_layer_us = [statistics.mean(e[i][0].elapsed_time(e[i][1]) for e in evs) * 1e3
+                    for i in range(len(W4_LAYERS))]
+
+    e2e = None
+    if not args.no_e2e:
+        def e2e_step():
+            for (wq, sc, ze, x, y), (xh, yh) in zip(layers, host):
+                x.copy_(xh, non_blocking=True)
+                G.gptq_w4a16_matmul(wq, sc, ze, cfg, x, Y=y)
+                yh.copy_(y, non_blocking=True)
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        ems = max_over_ranks(a.elapsed_time(b) / steps, world, dev)
+        e2e = {"value": world * step_bytes / (ems / 1e3) / 1e9, "unit": "GB/s", "ms_per_step": ems,
+               "h2d_bytes_per_step": sum(batch * dc * 2 for _, _, dc in W4_LAYERS),
+               "d2h_bytes_per_step": sum(batch * dr * 4 for _, dr, _ in W4_LAYERS)}
+    if rank != 0:
+        return
+    peaks, peak_src = load_peaks()
+    peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    big = max(range(len(W4_LAYERS)), key=lambda i: per_layer_us[i])
+    achieved = layer_bytes[big] / (per_layer_us[big] / 1e6) / 1e9
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        import numpy as np
+
+        from oracle import gptq_oracle as O
+        name, dr, dc = W4_LAYERS[1]
+        rows = 512
+        wq, sc, ze, _, _ = layers[1]
+        wh, sch, zeh = (wq[:rows].cpu().numpy().view(np.uint32), sc[:rows].cpu().numpy(),
+                        ze[:rows].cpu().numpy())
+        xf = host[1][0].float().numpy()
+        t = time.perf_counter()
+        O.dequantized_matmul(wh, sch, zeh, xf, 4, group)
+        sec = (time.perf_counter() - t) * dr / rows * len(W4_LAYERS)
+        cpu = {"value": step_bytes / sec / 1e9, "unit": "GB/s", "cores": cpu_cores(),
+               "kind": "oracle",
+               "sample": f"{name} rows 0..{rows - 1} of {dr} (x{dr / rows:g}), x3 layers"}
+    line = {
+        "metric": W4_METRIC, "value": world * step_bytes / (ms / 1e3) / 1e9, "unit": "GB/s",
+        "n_gpus": world, "steps": steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "u4 weights, bf16 activations, f32 accumulate", "data": "synthetic",
+        "config": {"workload": f"LLaMA-65B MLP (gate, up 22016x8192; down 8192x22016), "
+                               f"4-bit {f'g{group}' if group else 'per channel'}, batch {batch}",
+                   "batch": batch, "l2": "inputs larger than L2 (271 MB of packed layers per step)",
+                   "parallelism": f"{world} independent replica(s), one per GPU"},
+        "per_layer_us": dict(zip([n for n, _, _ in W4_LAYERS], per_layer_us)),
+        "roofline": {"bound": "hbm", "kernel": f"w4a16_matmul_kernel ({W4_LAYERS[big][0]})",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": kernel_traffic(f"w4a16_matmul_kernel/{W4_LAYERS[big][0]}",
+                                               "post_weight_quantization_26_b200/csrc/w4a16.cuh"),
+                     "algorithmic_bytes": layer_bytes[big],
+                     "peak_source": f"hbm_gbs of {peak_src}"},
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+
 
 def main():
     args = parse_args()
@@ -476,7 +617,10 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        run_ours(args, rank, world, local_rank)
+        if args.w4a16:
+            run_w4a16(args, rank, world, local_rank)
+        else:
+            run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:
             dist.destroy_process_group()

@@ -190,6 +190,28 @@ gptq_status gptq_dequant_check_noalloc(const uint32_t* qweight, const float* sca
                                        const gptq_config* cfg, float* W_hat,
                                        double* loss, void* stream);
 
+/* Y = X W^T with the packed layer dequantized on the fly (dingiv.github.io
+ * "量化" page, section GPTQ: the quantized weights serve inference, where
+ * batch-1 decoding is memory-bound and 4-bit weights cut the bytes read):
+ *   Y[b][r] = sum_k X[b][k] * s[r][g(k)] * (q[r][k] - z[r][g(k)]).
+ *  qweight, scales, zeros  the output of gptq_quantize_layer for a
+ *             d_row x d_col layer with cfg (device, read-only): qweight
+ *             16-byte aligned, scales 4-byte aligned, zero points 0..15.
+ *             cfg->bits must be 4; group_size as in the quantize call.
+ *  X          bf16 batch x d_col, row-major, 16-byte aligned (device).
+ *  batch      1 to 8 activation rows.
+ *  Y          fp32 batch x d_row, row-major (device, every element written).
+ * The products (q - z) x are formed exactly and summed in fp32 (tensor-core
+ * accumulation), so |Y - exact| <= (8 ceil(d_col / 1024) + 32) 2^-23
+ * sum_k |X[b][k]| |W^[r][k]|.
+ * Asynchronous on `stream`; allocates nothing.  Returns GPTQ_ERR_INVALID for
+ * other widths, batches, misaligned pointers or a d_col that is not a
+ * multiple of 32; nothing is launched then. */
+gptq_status gptq_w4a16_matmul(const uint32_t* qweight, const float* scales,
+                              const uint8_t* zeros, int64_t d_row, int64_t d_col,
+                              const gptq_config* cfg, const void* X, int64_t batch,
+                              float* Y, void* stream);
+
 /* Synchronize `stream`, then return and clear the device status word that
  * kernels set when a bounded internal wait runs out (GPTQ_ERR_TIMEOUT). */
 gptq_status gptq_device_status(void* stream);

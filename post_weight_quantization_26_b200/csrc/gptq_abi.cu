@@ -20,6 +20,7 @@
 #include "quantize.cuh"
 #include "syrk_tcgen05.cuh"
 #include "trailing_tf32.cuh"
+#include "w4a16.cuh"
 
 namespace {
 
@@ -86,6 +87,14 @@ gptq_status device_setup(int* num_sms) {
   DeviceInfo& di = g_dev[dev];
   if (!di.ready) {
     GPTQ_CUDA_TRY(cudaDeviceGetAttribute(&di.num_sms, cudaDevAttrMultiProcessorCount, dev));
+    for (const void* f : {reinterpret_cast<const void*>(w4a16::w4a16_matmul_kernel<0, 1>),
+                          reinterpret_cast<const void*>(w4a16::w4a16_matmul_kernel<0, 2>),
+                          reinterpret_cast<const void*>(w4a16::w4a16_matmul_kernel<4, 1>),
+                          reinterpret_cast<const void*>(w4a16::w4a16_matmul_kernel<4, 2>),
+                          reinterpret_cast<const void*>(w4a16::w4a16_matmul_kernel<2, 1>),
+                          reinterpret_cast<const void*>(w4a16::w4a16_matmul_kernel<1, 1>)})
+      GPTQ_CUDA_TRY(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         w4a16::WARPS * w4a16::WARP_BUDGET + w4a16::RED_BYTES));
     GPTQ_CUDA_TRY(cudaFuncSetAttribute(syrk::syrk_bf16_tcgen05_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        syrk::SMEM_BYTES));
@@ -298,6 +307,54 @@ size_t gptq_workspace_size(int64_t d_row, int64_t d_col, const gptq_config* cfg)
   const size_t b = quant_layout(d_row, d_col, cfg->block).total;
   const size_t c = check_layout(d_row, d_col).total;
   return std::max(a, std::max(b, c));
+}
+
+gptq_status gptq_w4a16_matmul(const uint32_t* qweight, const float* scales,
+                              const uint8_t* zeros, int64_t d_row, int64_t d_col,
+                              const gptq_config* cfg, const void* X, int64_t batch,
+                              float* Y, void* stream) {
+  if (!qweight || !scales || !zeros || !X || !Y) return GPTQ_ERR_INVALID;
+  if (d_row < 1 || d_row > (int64_t(1) << 24) || d_col < 32 || d_col % 32 != 0 ||
+      d_col > 65536)
+    return GPTQ_ERR_INVALID;
+  if (!config_ok(cfg, d_col) || cfg->bits != 4) return GPTQ_ERR_INVALID;
+  if (batch < 1 || batch > 8 || !aligned(X, 16) || !aligned(qweight, 16) || !aligned(scales, 4) ||
+      !aligned(Y, 4))
+    return GPTQ_ERR_INVALID;
+  int num_sms = 148;
+  gptq_status st = device_setup(&num_sms);
+  if (st != GPTQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int dr = static_cast<int>(d_row), dc = static_cast<int>(d_col), nb = static_cast<int>(batch);
+  const int g = cfg->group_size, n_groups = g ? dc / g : 1;
+  const int tiles = (dr + w4a16::ROWS - 1) / w4a16::ROWS;
+  // two 128-column chunks per work item where the scale regions are whole
+  // chunks and the activations leave room for a deep ring; one otherwise
+  const int cpi = (g == 0 || g % 128 == 0) && nb <= 4 ? 2 : 1;
+  const int depth = w4a16::ring_depth(cpi, nb), smem = w4a16::smem_bytes(cpi, nb);
+  const int per_sm = std::max(1, std::min(2, (228 * 1024) / (smem + 1024)));
+  const int grid = std::min(tiles, per_sm * num_sms);  // persistent CTAs
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(X);
+  // ceil(2^32 / group): umulhi(k, gmagic) == k / group for k, group < 2^16
+  const uint32_t gmagic = g ? static_cast<uint32_t>(((uint64_t(1) << 32) + g - 1) / g) : 0u;
+#define GPTQ_W4(GJ, CPI)                                                                   \
+  w4a16::w4a16_matmul_kernel<GJ, CPI><<<grid, w4a16::THREADS, smem, s>>>(                  \
+      qweight, scales, zeros, xb, Y, dr, dc, nb, gmagic, n_groups, depth)
+  // a scale region of 32 GJ columns must lie inside one group
+  if (g == 0) {
+    if (cpi == 2) GPTQ_W4(0, 2);
+    else GPTQ_W4(0, 1);
+  } else if (g % 128 == 0) {
+    if (cpi == 2) GPTQ_W4(4, 2);
+    else GPTQ_W4(4, 1);
+  } else if (g % 64 == 0) {
+    GPTQ_W4(2, 1);
+  } else {
+    GPTQ_W4(1, 1);
+  }
+#undef GPTQ_W4
+  GPTQ_LAUNCH_CHECK();
+  return GPTQ_OK;
 }
 
 gptq_status gptq_device_status(void* stream) {

@@ -25,7 +25,7 @@ STATUS_NAMES = {0: "GPTQ_OK", 1: "GPTQ_ERR_INVALID", 2: "GPTQ_ERR_NOT_SPD",
 EXPORTED = ("gptq_workspace_size", "gptq_hessian_accumulate",
             "gptq_prepare_hinv", "gptq_quantize_layer", "gptq_dequant_check",
             "gptq_device_status", "gptq_status_string", "gptq_launch_count",
-            "gptq_dequant_check_noalloc")
+            "gptq_dequant_check_noalloc", "gptq_w4a16_matmul")
 NOALLOC_MAX_TILES = 65536  # GPTQ_NOALLOC_MAX_TILES in include/gptq.h
 
 
@@ -78,6 +78,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gptq_dequant_check_noalloc.argtypes = [P, P, P, P, P, I64, I64, cfgp, P,
                                                ctypes.POINTER(D), P]
     lib.gptq_dequant_check_noalloc.restype = I
+    lib.gptq_w4a16_matmul.argtypes = [P, P, P, I64, I64, cfgp, P, I64, P, P]
+    lib.gptq_w4a16_matmul.restype = I
     lib.gptq_device_status.argtypes = [P]
     lib.gptq_device_status.restype = I
     lib.gptq_launch_count.argtypes = []
@@ -189,6 +191,24 @@ def gptq_dequant_check_noalloc(qweight, scales, zeros, W, H, cfg: GptqConfig,
         ctypes.byref(loss) if want_loss else None, _stream(stream))
     _check(st, "gptq_dequant_check_noalloc")
     return loss.value if want_loss else None
+
+
+def gptq_w4a16_matmul(qweight, scales, zeros, cfg: GptqConfig, X, Y=None,
+                      stream=None):
+    """Y = X W^T for bf16 X (batch x d_col, batch 1..8) and the packed 4-bit
+    layer (qweight, scales, zeros) as gptq_quantize_layer wrote it.  Y is fp32
+    batch x d_row, allocated here when not given.  Returns Y."""
+    assert X.dtype == torch.bfloat16 and X.dim() == 2 and X.is_contiguous()
+    batch, d_col = X.shape
+    d_row = scales.shape[0]
+    if Y is None:
+        Y = torch.empty(batch, d_row, dtype=torch.float32, device=X.device)
+    assert Y.dtype == torch.float32 and Y.shape == (batch, d_row) and Y.is_contiguous()
+    st = load_library().gptq_w4a16_matmul(
+        _ptr(qweight), _ptr(scales), _ptr(zeros), d_row, d_col,
+        ctypes.byref(cfg), _ptr(X), batch, _ptr(Y), _stream(stream))
+    _check(st, "gptq_w4a16_matmul")
+    return Y
 
 
 def gptq_device_status(stream=None) -> int:

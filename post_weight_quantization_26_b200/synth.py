@@ -230,3 +230,27 @@ def tiny_spec(d_row: int, d_col: int, n_tokens: int, seed: int = 0,
     return SMALL_256.with_(name=f"tiny_{d_row}x{d_col}_t{n_tokens}",
                            d_row=d_row, d_col=d_col, n_tokens=n_tokens,
                            w_seed=seed, x_seed=seed, **kw)
+
+
+def gen_packed_layer(d_row: int, d_col: int, group: int, seed: int = 0):
+    """A random 4-bit packed layer in the quantizer's output format, as CPU
+    tensors: ``words`` int32 ``[d_row][d_col/8]`` (uniform random bits, so
+    every code 0..15 is equally likely), ``scales`` fp32 ``[d_row][n_groups]``
+    drawn as ``0.002 + 0.01 |N(0,1)|``, ``zeros`` uint8 ``[d_row][n_groups]``
+    uniform in 0..15.  Stands in for a quantized layer where only the format
+    matters (the dequantized matmul), so no GPTQ run is needed at full size."""
+    assert d_col % 8 == 0
+    ng = 1 if group == 0 else d_col // group
+    g = torch.Generator().manual_seed(seed * 1000003 + 4242)
+    words = torch.randint(-(1 << 31), 1 << 31, (d_row, d_col // 8),
+                          generator=g, dtype=torch.int64).to(torch.int32)
+    scales = 0.002 + 0.01 * torch.randn((d_row, ng), generator=g).abs()
+    zeros = torch.randint(0, 16, (d_row, ng), generator=g, dtype=torch.uint8)
+    return words.contiguous(), scales.contiguous(), zeros.contiguous()
+
+
+def gen_activations(batch: int, d_col: int, seed: int = 0) -> torch.Tensor:
+    """``batch`` activation rows ``[batch][d_col]`` bf16 with N(0,1) entries
+    (the decoding-time input of a quantized linear layer)."""
+    g = torch.Generator().manual_seed(seed * 1000003 + 777)
+    return torch.randn((batch, d_col), generator=g).to(torch.bfloat16)

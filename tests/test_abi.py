@@ -120,6 +120,28 @@ def test_prepare_and_quantize_validation(lib):
                                   1 << 20, None) == 1
 
 
+def test_w4a16_matmul_validation(lib):
+    """Rejected before any launch: other widths, batches, shapes, alignment."""
+    from post_weight_quantization_26_b200 import gptq as G
+    f = lib.gptq_w4a16_matmul
+    cfg4, cfg3 = G.make_config(bits=4), G.make_config(bits=3)
+    ok = (FAKE, FAKE, FAKE, 64, 256)
+    assert f(*ok, ctypes.byref(cfg3), FAKE, 1, FAKE, None) == 1   # width 3
+    assert f(*ok, ctypes.byref(cfg4), FAKE, 0, FAKE, None) == 1   # batch 0
+    assert f(*ok, ctypes.byref(cfg4), FAKE, 9, FAKE, None) == 1   # batch 9
+    assert f(FAKE, FAKE, FAKE, 64, 48, ctypes.byref(cfg4), FAKE, 1, FAKE,
+             None) == 1                                            # d_col % 32
+    assert f(FAKE, FAKE, FAKE, 0, 256, ctypes.byref(cfg4), FAKE, 1, FAKE,
+             None) == 1                                            # no rows
+    assert f(*ok, ctypes.byref(cfg4), ctypes.c_void_p(0x7F0000000008), 1,
+             FAKE, None) == 1                                      # X alignment
+    assert f(ctypes.c_void_p(0x7F0000000004), FAKE, FAKE, 64, 256,
+             ctypes.byref(cfg4), FAKE, 1, FAKE, None) == 1         # words alignment
+    assert f(*ok, ctypes.byref(cfg4), None, 1, FAKE, None) == 1   # null X
+    g100 = G.make_config(bits=4, group_size=100)
+    assert f(*ok, ctypes.byref(g100), FAKE, 1, FAKE, None) == 1   # group % 32
+
+
 def test_product_path_has_no_fallback():
     """The binding refuses to run without its library (no CPU path)."""
     from post_weight_quantization_26_b200 import gptq as G
