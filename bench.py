@@ -54,6 +54,9 @@ def parse_args():
                         "4-bit LLaMA-65B MLP layers with BATCH activation rows (1..8)")
     p.add_argument("--w4a16-group", type=int, default=128, metavar="G",
                    help="group size of the --w4a16 layers (0: one scale per output channel)")
+    p.add_argument("--shard-layer", action="store_true",
+                   help="strong scaling: ONE q_proj layer across the ranks (token-sharded H "
+                        "summed by an NCCL all-reduce, row-sharded quantize, rows gathered)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
@@ -601,6 +604,109 @@ def run_w4a16(args, rank, world, local_rank):
     }
     print(json.dumps(line), flush=True)
 
+# ------------------------------------------------- one layer across ranks
+def run_sharded(args, rank, world, local_rank):
+    """Strong scaling of one q_proj layer: rank r accumulates H over its
+    token shard, one NCCL all-reduce sums H, every rank factors it, and rank
+    r quantizes its row shard; the packed rows are gathered in rank order.
+    Value = the layer's weights / the slowest rank's step time."""
+    import torch
+    import torch.distributed as dist
+
+    from post_weight_quantization_26_b200 import build as _build
+    from post_weight_quantization_26_b200 import gptq as G
+    from post_weight_quantization_26_b200 import sharded, synth
+
+    if rank == 0:
+        _build.build()
+    if world > 1:
+        dist.barrier()
+    G.load_library()
+    dev = torch.device("cuda", local_rank)
+    spec = synth.Q_PROJ_7B  # the same layer on every rank
+    if args.tokens:
+        spec = spec.with_(n_tokens=args.tokens, name=f"{spec.name}_n{args.tokens}")
+    d, dr = spec.d_col, spec.d_row
+    t0, t1 = sharded.shard(spec.n_tokens, world, rank)
+    r0, r1 = sharded.shard(dr, world, rank)
+    cfg = G.make_config(bits=spec.bits, group_size=spec.group, sym=spec.sym,
+                        block=spec.block, damp_rel=spec.damp)
+    x = synth.gen_tokens(spec, t0, t1).to(dev)
+    w = synth.gen_weight(spec)[r0:r1].contiguous().to(dev)
+    stream = torch.cuda.current_stream(dev)
+    base = sharded.cuda_steps(cfg, spec.damp, world, dev)
+    marks = {}
+
+    def timed(name, fn):
+        def run(*a):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            out = fn(*a)
+            e1.record(stream)
+            marks.setdefault(name, []).append((e0, e1))
+            return out
+        return run
+
+    steps = sharded.Steps(base.zeros_h, timed("hessian", base.accumulate),
+                          timed("allreduce", base.allreduce_sum), timed("prepare", base.prepare),
+                          timed("quantize", base.quantize), timed("gather", base.allgather_rows))
+
+    def step():
+        return sharded.quantize_layer_sharded(steps, x, w, d)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    if G.gptq_device_status() != 0:
+        raise RuntimeError("device status set during warm-up")
+    marks.clear()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    launches0 = G.gptq_launch_count()
+    a.record(stream)
+    for _ in range(args.steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    launches = G.gptq_launch_count() - launches0
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    ms = max_over_ranks(a.elapsed_time(b) / args.steps, world, dev)
+    stage_ms = {k: statistics.mean(e0.elapsed_time(e1) for e0, e1 in v) for k, v in marks.items()}
+    if G.gptq_device_status() != 0:
+        raise RuntimeError("device status set during the timed region")
+    if rank != 0:
+        return
+    peaks, peak_src = load_peaks()
+    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    achieved = d * (d + 1) * (t1 - t0) / (stage_ms["hessian"] / 1e3) / 1e12
+    line = {
+        "metric": METRIC, "value": dr * d / (ms / 1e3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+        "dtype": "bf16 in / f32 acc (H); f64 (factor); f32 (sweep)",
+        "data": "synthetic (seeded LLaMA-7B-shaped layer and activations)",
+        "config": {"workload": f"{spec.name}, one layer across {world} GPU(s)",
+                   "d_row": dr, "d_col": d, "n_tokens": spec.n_tokens,
+                   "tokens_on_rank0": t1 - t0, "rows_on_rank0": r1 - r0,
+                   "l2": "inputs larger than L2 (X bf16 %.2f GB over all ranks)"
+                         % (spec.n_tokens * d * 2 / 1e9),
+                   "parallelism": "token-sharded H + NCCL all-reduce, row-sharded quantize, "
+                                  "rows all-gathered"},
+        "stage_ms_rank0": stage_ms,
+        "roofline": {"bound": "tensor", "kernel": "syrk_bf16_tcgen05_kernel (rank 0's tokens)",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "peak_source": f"bf16_tflops_sustained of {peak_src}"},
+        "cpu_baseline": None, "e2e": None, "gpu_launches": launches, "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+
 
 def main():
     args = parse_args()
@@ -619,6 +725,8 @@ def main():
     try:
         if args.w4a16:
             run_w4a16(args, rank, world, local_rank)
+        elif args.shard_layer:
+            run_sharded(args, rank, world, local_rank)
         else:
             run_ours(args, rank, world, local_rank)
     finally:
