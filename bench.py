@@ -57,6 +57,9 @@ def parse_args():
     p.add_argument("--shard-layer", action="store_true",
                    help="strong scaling: ONE q_proj layer across the ranks (token-sharded H "
                         "summed by an NCCL all-reduce, row-sharded quantize, rows gathered)")
+    p.add_argument("--awq", action="store_true",
+                   help="time the AWQ scale search (20-point alpha grid) on the q_proj layer "
+                        "with 32768 calibration tokens, 4-bit g128")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
@@ -707,6 +710,162 @@ def run_sharded(args, rank, world, local_rank):
     }
     print(json.dumps(line), flush=True)
 
+# ------------------------------------------------------ AWQ scale search
+AWQ_METRIC = "AWQ scale search: weights quantized/s per linear layer"
+AWQ_TOKENS = 32768  # the AWQ section's calibration size (~32K tokens)
+
+
+def run_awq(args, rank, world, local_rank):
+    """One step = the AWQ search for one q_proj layer: the channel scale and
+    the Hessian over 32768 calibration tokens, the 20-point alpha grid (each
+    point: quantize W diag(s), form dW, the output error through H) and the
+    4-bit quantization at the best alpha.  Each rank searches its own layer
+    (weak scaling, no collective)."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from post_weight_quantization_26_b200 import build as _build
+    from post_weight_quantization_26_b200 import gptq as G
+    from post_weight_quantization_26_b200 import synth
+
+    if rank == 0:
+        _build.build()
+    if world > 1:
+        dist.barrier()
+    G.load_library()
+    dev = torch.device("cuda", local_rank)
+    spec = workload_spec("q_proj", rank).with_(n_tokens=args.tokens or AWQ_TOKENS, group=128)
+    d, n, dr = spec.d_col, spec.n_tokens, spec.d_row
+    n_grid = 20
+    cfg = G.make_config(bits=4, group_size=128)
+    x_host = synth.gen_tokens(spec).pin_memory()
+    w_host = synth.gen_weight(spec).pin_memory()
+    x, w = x_host.to(dev), w_host.to(dev)
+    H = torch.zeros((d, d), dtype=torch.float32, device=dev)
+    sx = torch.empty(d, dtype=torch.float64, device=dev)
+    ws = torch.empty(G.gptq_awq_workspace_size(dr, d, cfg), dtype=torch.uint8, device=dev)
+    qw, sc, ze = G.alloc_outputs(dr, d, cfg, device=dev)
+    out = (torch.empty(n_grid, dtype=torch.float64, device=dev),
+           torch.empty(1, dtype=torch.int32, device=dev),
+           torch.empty(d, dtype=torch.float32, device=dev), qw, sc, ze)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        G.gptq_awq_channel_scale(x, sx)
+        H.zero_()
+        G.gptq_hessian_accumulate(H, x)
+        if ev:
+            ev[1].record(stream)
+        G.gptq_awq_search(w, H, sx, cfg, n_grid, ws=ws, out=out)
+        if ev:
+            ev[2].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    if G.gptq_device_status() != 0:
+        raise RuntimeError("device status set during warm-up")
+    steps = max(1, args.steps)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    launches0 = G.gptq_launch_count()
+    a.record(stream)
+    for i in range(steps):
+        step(evs[i])
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    launches = G.gptq_launch_count() - launches0
+    clk = clocks.stop()
+    ms = max_over_ranks(a.elapsed_time(b) / steps, world, dev)
+    stats_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    search_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    if G.gptq_device_status() != 0:
+        raise RuntimeError("device status set during the timed region")
+    best = int(out[1].item())
+
+    e2e = None
+    if not args.no_e2e:
+        qh = torch.empty(qw.shape, dtype=qw.dtype).pin_memory()
+        sh = torch.empty(sc.shape, dtype=sc.dtype).pin_memory()
+        zh = torch.empty(ze.shape, dtype=ze.dtype).pin_memory()
+        s_h = torch.empty(d, dtype=torch.float32).pin_memory()
+
+        def e2e_step():
+            x.copy_(x_host, non_blocking=True)
+            w.copy_(w_host, non_blocking=True)
+            step()
+            qh.copy_(qw, non_blocking=True)
+            sh.copy_(sc, non_blocking=True)
+            zh.copy_(ze, non_blocking=True)
+            s_h.copy_(out[2], non_blocking=True)
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ems = max_over_ranks(e0.elapsed_time(e1) / steps, world, dev)
+        e2e = {"value": world * dr * d / (ems / 1e3), "unit": UNIT, "ms_per_step": ems,
+               "h2d_bytes_per_step": n * d * 2 + dr * d * 4,
+               "d2h_bytes_per_step": qw.numel() * 4 + sc.numel() * 4 + ze.numel() + d * 4}
+    if rank != 0:
+        return
+    peaks, peak_src = load_peaks()
+    tf32_peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]) * (1.1 / 2.25)
+    tensor_flops = n_grid * 6.0 * dr * d * d  # three TF32 products of dW H per alpha
+    achieved = tensor_flops / (search_ms / 1e3) / 1e12
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        from oracle import awq_oracle as A
+        from oracle import gptq_oracle as O
+        rows, toks = 64, 8192
+        t0 = time.perf_counter()
+        xs = x_host[:toks].float().numpy()
+        sx_c = A.channel_scale(xs)
+        h_c = O.hessian(xs)
+        t1 = time.perf_counter()
+        A.search(w_host[:rows].numpy().astype(np.float64), h_c, sx_c, 4, 128, n_grid)
+        t2 = time.perf_counter()
+        sec = (t1 - t0) * n / toks + (t2 - t1) * dr / rows
+        cpu = {"value": dr * d / sec, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+               "sample": f"channel scale and H on {toks} of {n} tokens (x{n / toks:g}); the "
+                         f"20-point search on {rows} of {dr} rows (x{dr / rows:g})"}
+    line = {
+        "metric": AWQ_METRIC, "value": world * dr * d / (ms / 1e3), "unit": UNIT, "n_gpus": world,
+        "steps": steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 in / f32 acc (H); split-TF32 (dW H); f64 (loss sums)",
+        "data": "synthetic (seeded LLaMA-7B-shaped layer and activations)",
+        "config": {"workload": f"AWQ {spec.name} 4096x4096, {n} tokens, 4-bit g128, "
+                               f"{n_grid}-point alpha grid",
+                   "d_row": dr, "d_col": d, "n_tokens": n, "group_size": 128, "n_grid": n_grid,
+                   "l2": "inputs larger than L2 (X bf16 %.2f GB; dW splits and T 192 MB per "
+                         "alpha)" % (n * d * 2 / 1e9),
+                   "parallelism": f"{world} independent layer(s), one per GPU"},
+        "stage_ms": {"channel_scale_and_hessian": stats_ms, "search": search_ms},
+        "best_alpha": best / (n_grid - 1),
+        "roofline": {"bound": "tensor", "kernel": "trailing_tf32x3_kernel (dW H), over the "
+                                                  "whole search stage",
+                     "achieved": achieved, "peak": tf32_peak, "unit": "TFLOP/s",
+                     "frac": achieved / tf32_peak, "traffic": None,
+                     "peak_source": f"bf16_tflops_sustained of {peak_src} x 1.1/2.25 "
+                                    "(nominal tf32/bf16)"},
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+
 
 def main():
     args = parse_args()
@@ -727,6 +886,8 @@ def main():
             run_w4a16(args, rank, world, local_rank)
         elif args.shard_layer:
             run_sharded(args, rank, world, local_rank)
+        elif args.awq:
+            run_awq(args, rank, world, local_rank)
         else:
             run_ours(args, rank, world, local_rank)
     finally:

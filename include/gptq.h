@@ -212,6 +212,54 @@ gptq_status gptq_w4a16_matmul(const uint32_t* qweight, const float* scales,
                               const gptq_config* cfg, const void* X, int64_t batch,
                               float* Y, void* stream);
 
+/* AWQ channel scale (dingiv.github.io "量化" page, section AWQ: salient
+ * input channels are found by their mean activation magnitude):
+ *   sx[k] = (1/n) sum_t |X[t][k]|.
+ *  X    bf16 calibration tokens, token-major: token t at X + t*ldx
+ *       (device, 16-byte aligned; ldx >= d, ldx % 8 == 0).
+ *  n    tokens, >= 1.   d  channels, a multiple of 8, <= 65536.
+ *  sx   fp64[d] (device, written).  The sums are exact in fp64 for bf16
+ *       inputs, so the result does not depend on the order of summation.
+ * Asynchronous on `stream`.  GPTQ_ERR_INVALID for bad sizes or pointers. */
+gptq_status gptq_awq_channel_scale(const void* X, int64_t n, int64_t d, int64_t ldx, double* sx,
+                                   void* stream);
+
+/* Workspace bytes for gptq_awq_search: 2 d_col^2 + 3 d_row d_col floats and a
+ * few KB.  0 for an unsupported configuration. */
+size_t gptq_awq_workspace_size(int64_t d_row, int64_t d_col, const gptq_config* cfg);
+
+/* AWQ scale search (dingiv.github.io "量化" page, section AWQ): for each
+ * alpha_a = a / (n_grid - 1), s = sx^alpha (s = 1 where sx = 0), W diag(s)
+ * is quantized to 4 bits with the min-max quantizer of this library and
+ * divided by s again, and the loss is the layer's output error
+ *   L(alpha) = ||W X - Q(W diag(s)) diag(s)^-1 X||_F^2
+ *            = 1/2 sum_r dW_r H dW_r^T,   H = 2 X X^T.
+ * The best alpha (the first smallest loss) is then applied: the outputs are
+ * the codes, scales and zero points of W diag(s*) and s* itself (the
+ * activations, or the previous layer's output, are divided by s*).
+ *  W        fp32 d_row x d_col, row-major (device, 16-byte aligned, read).
+ *  H        fp32 d_col x d_col upper triangle as gptq_hessian_accumulate
+ *           writes it (device, 16-byte aligned, read).
+ *  sx       fp64[d_col] from gptq_awq_channel_scale (device).
+ *  cfg      bits 4, sym 0, group_size 0 (one scale per row) or a multiple of
+ *           32 dividing d_col; d_col a multiple of 32, <= 65536.
+ *  n_grid   grid points, 2 to 64 (the AWQ section uses 20).
+ *  losses   fp64[n_grid] (device, written): L(alpha_a).
+ *  best     int32 (device, written): a of the best alpha.
+ *  s_out    fp32[d_col] (device, written): s*.
+ *  qweight, scales, zeros  as written by gptq_quantize_layer for 4 bits
+ *           (device, written), here for W diag(s*).
+ *  ws       >= gptq_awq_workspace_size bytes (device, 256-byte aligned).
+ * The contraction dW H runs on the tensor cores as three TF32 products of
+ * hi/lo splits (about fp32 accuracy); the loss is summed in fp64.
+ * Asynchronous on `stream`; allocates nothing.  GPTQ_ERR_INVALID for bad
+ * sizes, configurations or pointers, GPTQ_ERR_WORKSPACE for a short or
+ * misaligned workspace; nothing is launched then. */
+gptq_status gptq_awq_search(const float* W, const float* H, const double* sx, int64_t d_row,
+                            int64_t d_col, const gptq_config* cfg, int n_grid, double* losses,
+                            int32_t* best, float* s_out, uint32_t* qweight, float* scales,
+                            uint8_t* zeros, void* ws, size_t ws_bytes, void* stream);
+
 /* Synchronize `stream`, then return and clear the device status word that
  * kernels set when a bounded internal wait runs out (GPTQ_ERR_TIMEOUT). */
 gptq_status gptq_device_status(void* stream);

@@ -21,6 +21,7 @@
 #include "syrk_tcgen05.cuh"
 #include "trailing_tf32.cuh"
 #include "w4a16.cuh"
+#include "awq.cuh"
 
 namespace {
 
@@ -206,6 +207,30 @@ CheckWs check_layout(int64_t d_row, int64_t d_col) {
   return w;
 }
 
+// ------------------------------------------------------------------ AWQ
+struct AwqWs {
+  size_t Hhi, Hlo, Ehi, Elo, T, s, partials, total;
+};
+AwqWs awq_layout(int64_t d_row, int64_t d_col) {
+  AwqWs w{};
+  size_t off = 0;
+  const size_t hh = static_cast<size_t>(d_col) * d_col * 4, ww = static_cast<size_t>(d_row) * d_col * 4;
+  w.Hhi = off; off = align_up(off + hh);
+  w.Hlo = off; off = align_up(off + hh);
+  w.Ehi = off; off = align_up(off + ww);
+  w.Elo = off; off = align_up(off + ww);
+  w.T = off; off = align_up(off + ww);
+  w.s = off; off = align_up(off + static_cast<size_t>(d_col) * 4);
+  w.partials = off; off = align_up(off + awq::DOT_BLOCKS * 8);
+  w.total = off;
+  return w;
+}
+
+bool awq_config_ok(const gptq_config* cfg, int64_t d_row, int64_t d_col) {
+  return config_ok(cfg, d_col) && cfg->bits == 4 && cfg->sym == 0 && d_row >= 1 &&
+         d_row <= (int64_t(1) << 24) && d_col >= 32 && d_col % 32 == 0 && d_col <= 65536;
+}
+
 // 2D fp32 tensor map: dims {inner, outer}, row stride in elements, box {bx, by}.
 gptq_status encode_f32_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer,
                           uint64_t row_stride, uint32_t bx, uint32_t by,
@@ -353,6 +378,103 @@ gptq_status gptq_w4a16_matmul(const uint32_t* qweight, const float* scales,
     GPTQ_W4(1, 1);
   }
 #undef GPTQ_W4
+  GPTQ_LAUNCH_CHECK();
+  return GPTQ_OK;
+}
+
+gptq_status gptq_awq_channel_scale(const void* X, int64_t n, int64_t d, int64_t ldx, double* sx,
+                                   void* stream) {
+  if (!X || !sx) return GPTQ_ERR_INVALID;
+  if (n < 1 || n > (int64_t(1) << 31) - 1 || d < 8 || d % 8 != 0 || d > 65536) return GPTQ_ERR_INVALID;
+  if (ldx < d || ldx % 8 != 0 || !aligned(X, 16) || !aligned(sx, 8)) return GPTQ_ERR_INVALID;
+  int num_sms = 148;
+  gptq_status st = device_setup(&num_sms);
+  if (st != GPTQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int dn = static_cast<int>(d), nn = static_cast<int>(n);
+  GPTQ_CUDA_TRY(cudaMemsetAsync(sx, 0, static_cast<size_t>(d) * 8, s));
+  const int tpb = std::max(256, (nn + 65534) / 65535);  // tokens per block (grid.y <= 65535)
+  const dim3 grid((dn + awq::COLS_PER_BLOCK - 1) / awq::COLS_PER_BLOCK, (nn + tpb - 1) / tpb);
+  awq::absum_kernel<<<grid, awq::THREADS, 0, s>>>(static_cast<const __nv_bfloat16*>(X), nn, dn,
+                                                  ldx, tpb, sx);
+  GPTQ_LAUNCH_CHECK();
+  awq::mean_kernel<<<(dn + 255) / 256, 256, 0, s>>>(sx, dn, nn);
+  GPTQ_LAUNCH_CHECK();
+  return GPTQ_OK;
+}
+
+size_t gptq_awq_workspace_size(int64_t d_row, int64_t d_col, const gptq_config* cfg) {
+  if (!awq_config_ok(cfg, d_row, d_col)) return 0;
+  return awq_layout(d_row, d_col).total;
+}
+
+gptq_status gptq_awq_search(const float* W, const float* H, const double* sx, int64_t d_row,
+                            int64_t d_col, const gptq_config* cfg, int n_grid, double* losses,
+                            int32_t* best, float* s_out, uint32_t* qweight, float* scales,
+                            uint8_t* zeros, void* ws, size_t ws_bytes, void* stream) {
+  if (!W || !H || !sx || !losses || !best || !s_out || !qweight || !scales || !zeros)
+    return GPTQ_ERR_INVALID;
+  if (!awq_config_ok(cfg, d_row, d_col) || n_grid < 2 || n_grid > 64) return GPTQ_ERR_INVALID;
+  if (!aligned(W, 16) || !aligned(H, 16) || !aligned(sx, 8) || !aligned(losses, 8) ||
+      !aligned(best, 4) || !aligned(s_out, 4) || !aligned(qweight, 4) || !aligned(scales, 4))
+    return GPTQ_ERR_INVALID;
+  const AwqWs L = awq_layout(d_row, d_col);
+  if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return GPTQ_ERR_WORKSPACE;
+  int num_sms = 148;
+  gptq_status st = device_setup(&num_sms);
+  if (st != GPTQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  float* Hhi = reinterpret_cast<float*>(base + L.Hhi);
+  float* Hlo = reinterpret_cast<float*>(base + L.Hlo);
+  float* Ehi = reinterpret_cast<float*>(base + L.Ehi);
+  float* Elo = reinterpret_cast<float*>(base + L.Elo);
+  float* T = reinterpret_cast<float*>(base + L.T);
+  float* sv = reinterpret_cast<float*>(base + L.s);
+  double* partials = reinterpret_cast<double*>(base + L.partials);
+  const int dr = static_cast<int>(d_row), dc = static_cast<int>(d_col);
+  const int gw = cfg->group_size ? cfg->group_size : dc;
+  // the contraction T -= dW H on the split-TF32 tcgen05 kernel: E = dW
+  // (K-major, K = d_col), G = H (all d_col rows), output T
+  CUtensorMap tm_ehi, tm_elo, tm_hhi, tm_hlo, tm_t;
+  if ((st = encode_f32_2d(&tm_ehi, Ehi, dc, dr, dc, trail::BK, trail::BM, CU_TENSOR_MAP_SWIZZLE_64B)) != GPTQ_OK ||
+      (st = encode_f32_2d(&tm_elo, Elo, dc, dr, dc, trail::BK, trail::BM, CU_TENSOR_MAP_SWIZZLE_64B)) != GPTQ_OK ||
+      (st = encode_f32_2d(&tm_hhi, Hhi, dc, dc, dc, trail::B_BOX, trail::BK,
+                          CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B)) != GPTQ_OK ||
+      (st = encode_f32_2d(&tm_hlo, Hlo, dc, dc, dc, trail::B_BOX, trail::BK,
+                          CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B)) != GPTQ_OK ||
+      (st = encode_f32_2d(&tm_t, T, dc, dr, dc, trail::OUT_COLS, trail::BM, CU_TENSOR_MAP_SWIZZLE_128B)) != GPTQ_OK)
+    return st;
+  trail::Params tp{};
+  tp.M = dr; tp.N = dc; tp.K = dc; tp.n0 = 0; tp.j0 = 0;
+  tp.tiles_m = (dr + trail::BM - 1) / trail::BM;
+  tp.tiles_n = (dc + trail::BN - 1) / trail::BN;
+  tp.tiles = tp.tiles_m * tp.tiles_n;
+  const int tgrid = std::min(tp.tiles, num_sms);
+  const int units = dr * (dc / gw);
+  const int qgrid = std::max(1, std::min((units + 7) / 8, num_sms * 8));
+  const size_t nel = static_cast<size_t>(dr) * dc;
+
+  awq::sym_split_kernel<<<num_sms * 4, 256, 0, s>>>(H, dc, Hhi, Hlo);
+  GPTQ_LAUNCH_CHECK();
+  for (int a = 0; a < n_grid; ++a) {
+    const double alpha = static_cast<double>(a) / static_cast<double>(n_grid - 1);
+    awq::scales_kernel<<<(dc + 255) / 256, 256, 0, s>>>(sx, dc, alpha, sv);
+    GPTQ_LAUNCH_CHECK();
+    awq::delta_kernel<<<qgrid, awq::THREADS, 0, s>>>(W, sv, dr, dc, gw, Ehi, Elo);
+    GPTQ_LAUNCH_CHECK();
+    GPTQ_CUDA_TRY(cudaMemsetAsync(T, 0, nel * 4, s));
+    trail::trailing_tf32x3_kernel<<<tgrid, trail::NUM_THREADS, trail::SMEM_BYTES, s>>>(
+        tm_ehi, tm_elo, tm_hhi, tm_hlo, tm_t, tp);
+    GPTQ_LAUNCH_CHECK();
+    awq::dot_kernel<<<awq::DOT_BLOCKS, awq::THREADS, 0, s>>>(Ehi, Elo, T, nel / 4, partials);
+    GPTQ_LAUNCH_CHECK();
+    awq::finalize_kernel<<<1, 1024, 0, s>>>(partials, awq::DOT_BLOCKS, losses + a);
+    GPTQ_LAUNCH_CHECK();
+  }
+  awq::argmin_kernel<<<1, 256, 0, s>>>(losses, n_grid, sx, dc, best, s_out);
+  GPTQ_LAUNCH_CHECK();
+  awq::pack_kernel<<<qgrid, awq::THREADS, 0, s>>>(W, s_out, dr, dc, gw, qweight, scales, zeros);
   GPTQ_LAUNCH_CHECK();
   return GPTQ_OK;
 }

@@ -25,7 +25,8 @@ STATUS_NAMES = {0: "GPTQ_OK", 1: "GPTQ_ERR_INVALID", 2: "GPTQ_ERR_NOT_SPD",
 EXPORTED = ("gptq_workspace_size", "gptq_hessian_accumulate",
             "gptq_prepare_hinv", "gptq_quantize_layer", "gptq_dequant_check",
             "gptq_device_status", "gptq_status_string", "gptq_launch_count",
-            "gptq_dequant_check_noalloc", "gptq_w4a16_matmul")
+            "gptq_dequant_check_noalloc", "gptq_w4a16_matmul", "gptq_awq_channel_scale",
+            "gptq_awq_workspace_size", "gptq_awq_search")
 NOALLOC_MAX_TILES = 65536  # GPTQ_NOALLOC_MAX_TILES in include/gptq.h
 
 
@@ -80,6 +81,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gptq_dequant_check_noalloc.restype = I
     lib.gptq_w4a16_matmul.argtypes = [P, P, P, I64, I64, cfgp, P, I64, P, P]
     lib.gptq_w4a16_matmul.restype = I
+    lib.gptq_awq_channel_scale.argtypes = [P, I64, I64, I64, P, P]
+    lib.gptq_awq_channel_scale.restype = I
+    lib.gptq_awq_workspace_size.argtypes = [I64, I64, cfgp]
+    lib.gptq_awq_workspace_size.restype = SZ
+    lib.gptq_awq_search.argtypes = [P, P, P, I64, I64, cfgp, I, P, P, P, P, P, P, P, SZ, P]
+    lib.gptq_awq_search.restype = I
     lib.gptq_device_status.argtypes = [P]
     lib.gptq_device_status.restype = I
     lib.gptq_launch_count.argtypes = []
@@ -209,6 +216,48 @@ def gptq_w4a16_matmul(qweight, scales, zeros, cfg: GptqConfig, X, Y=None,
         ctypes.byref(cfg), _ptr(X), batch, _ptr(Y), _stream(stream))
     _check(st, "gptq_w4a16_matmul")
     return Y
+
+
+def gptq_awq_channel_scale(X, sx=None, stream=None):
+    """sx[k] = mean_t |X[t][k]| (fp64) for token-major bf16 X (n x d)."""
+    assert X.dtype == torch.bfloat16 and X.dim() == 2 and X.stride(1) == 1
+    n, d = X.shape
+    if sx is None:
+        sx = torch.empty(d, dtype=torch.float64, device=X.device)
+    st = load_library().gptq_awq_channel_scale(_ptr(X), n, d, X.stride(0), _ptr(sx),
+                                               _stream(stream))
+    _check(st, "gptq_awq_channel_scale")
+    return sx
+
+
+def gptq_awq_workspace_size(d_row: int, d_col: int, cfg: GptqConfig) -> int:
+    n = load_library().gptq_awq_workspace_size(d_row, d_col, ctypes.byref(cfg))
+    if n == 0:
+        raise GptqError(1, "gptq_awq_workspace_size")
+    return int(n)
+
+
+def gptq_awq_search(W, H, sx, cfg: GptqConfig, n_grid: int = 20, ws=None, out=None,
+                    stream=None):
+    """The AWQ grid search over alpha; returns (losses fp64[n_grid], best
+    int32[1], s fp32[d_col], qweight, scales, zeros), all on the device."""
+    d_row, d_col = W.shape
+    dev = W.device
+    if ws is None:
+        ws = torch.empty(gptq_awq_workspace_size(d_row, d_col, cfg), dtype=torch.uint8,
+                         device=dev)
+    if out is None:
+        qw, sc, ze = alloc_outputs(d_row, d_col, cfg, device=dev)
+        out = (torch.empty(n_grid, dtype=torch.float64, device=dev),
+               torch.empty(1, dtype=torch.int32, device=dev),
+               torch.empty(d_col, dtype=torch.float32, device=dev), qw, sc, ze)
+    losses, best, s, qw, sc, ze = out
+    st = load_library().gptq_awq_search(
+        _ptr(W), _ptr(H), _ptr(sx), d_row, d_col, ctypes.byref(cfg), int(n_grid), _ptr(losses),
+        _ptr(best), _ptr(s), _ptr(qw), _ptr(sc), _ptr(ze), _ptr(ws), ws.numel(),
+        _stream(stream))
+    _check(st, "gptq_awq_search")
+    return out
 
 
 def gptq_device_status(stream=None) -> int:

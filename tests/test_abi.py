@@ -142,6 +142,33 @@ def test_w4a16_matmul_validation(lib):
     assert f(*ok, ctypes.byref(g100), FAKE, 1, FAKE, None) == 1   # group % 32
 
 
+def test_awq_validation(lib):
+    """The AWQ entry points reject bad sizes, configurations and pointers
+    before anything is launched."""
+    from post_weight_quantization_26_b200 import gptq as G
+    g128, bad3, sym = G.make_config(bits=4, group_size=128), G.make_config(bits=3), \
+        G.make_config(bits=4, sym=True)
+    wsz = lib.gptq_awq_workspace_size
+    assert wsz(64, 256, ctypes.byref(g128)) >= 2 * 256 * 256 * 4 + 3 * 64 * 256 * 4
+    assert wsz(64, 256, ctypes.byref(bad3)) == 0          # AWQ is 4-bit only
+    assert wsz(64, 256, ctypes.byref(sym)) == 0           # asymmetric quantizer
+    assert wsz(64, 48, ctypes.byref(G.make_config(bits=4))) == 0  # d_col % 32
+    cs = lib.gptq_awq_channel_scale
+    assert cs(FAKE, 0, 64, 64, FAKE, None) == 1            # no tokens
+    assert cs(FAKE, 16, 12, 16, FAKE, None) == 1           # d % 8
+    assert cs(FAKE, 16, 64, 60, FAKE, None) == 1           # ldx < d
+    assert cs(ctypes.c_void_p(0x7F0000000008), 16, 64, 64, FAKE, None) == 1  # alignment
+    sr = lib.gptq_awq_search
+    args = [FAKE, FAKE, FAKE, 64, 256, ctypes.byref(g128)]
+    out = [FAKE] * 6
+    assert sr(*args, 1, *out, FAKE, 1 << 30, None) == 1    # n_grid < 2
+    assert sr(*args, 65, *out, FAKE, 1 << 30, None) == 1   # n_grid > 64
+    assert sr(*args, 20, *out, FAKE, 16, None) == 4        # short workspace
+    assert sr(*args, 20, *out, ctypes.c_void_p(0x7F0000000010), 1 << 30, None) == 4
+    assert sr(FAKE, FAKE, FAKE, 64, 256, ctypes.byref(bad3), 20, *out, FAKE, 1 << 30,
+              None) == 1
+
+
 def test_product_path_has_no_fallback():
     """The binding refuses to run without its library (no CPU path)."""
     from post_weight_quantization_26_b200 import gptq as G

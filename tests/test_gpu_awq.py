@@ -1,0 +1,122 @@
+"""GPU parity of the AWQ scale search (through the C ABI) against the AWQ
+oracle on the same seeded layers and calibration tokens.
+
+Bars: the channel scale is exact (fp64 sums of bf16 magnitudes); s* equals
+the oracle's s rounded to fp32; the codes and zero points of W diag(s*) are
+those of the oracle taking its decisions in fp32 (at most 0.1% of codes off
+by one, as for the GPTQ path); each alpha's loss is within 1e-4 relative of
+the oracle's.  The loss goes through the fp32 SYRK (H relative error ~1e-7)
+and a split-TF32 contraction (~1e-6 of the product), so 1e-4 leaves room.
+The chosen alpha is the oracle's, unless the two losses involved are within
+that same tolerance of each other.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import awq_oracle as A
+from oracle import gptq_oracle as O
+from post_weight_quantization_26_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+LOSS_RTOL = 1e-4
+
+
+@pytest.fixture(scope="module")
+def G():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    from post_weight_quantization_26_b200 import build, gptq
+    build.build()
+    gptq.load_library()
+    return gptq
+
+
+def _gpu_search(G, x_cpu, w_cpu, group, n_grid=20):
+    d = x_cpu.shape[1]
+    cfg = G.make_config(bits=4, group_size=group)
+    x, w = x_cpu.cuda(), w_cpu.cuda()
+    h = torch.zeros((d, d), dtype=torch.float32, device="cuda")
+    G.gptq_hessian_accumulate(h, x)
+    sx = G.gptq_awq_channel_scale(x)
+    losses, best, s, qw, sc, ze = G.gptq_awq_search(w, h, sx, cfg, n_grid)
+    torch.cuda.synchronize()
+    assert G.gptq_device_status() == 0
+    codes = O.unpack_codes(qw.cpu().numpy().view(np.uint32), 4, d)
+    return dict(sx=sx.cpu().numpy(), losses=losses.cpu().numpy(), best=int(best.item()),
+                s=s.cpu().numpy(), codes=codes, scales=sc.cpu().numpy(), zeros=ze.cpu().numpy(),
+                h=h)
+
+
+def _check_codes(c, ref, frac=1e-3):
+    diff = np.abs(c.astype(np.int64) - ref.astype(np.int64))
+    assert diff.max(initial=0) <= 1
+    assert np.mean(diff != 0) <= frac
+
+
+def _check_against_oracle(r, x, w, group):
+    xf = x.float().numpy().astype(np.float64)
+    wf = w.numpy().astype(np.float64)
+    sx = A.channel_scale(xf)
+    np.testing.assert_array_equal(r["sx"], sx)
+    ref = A.search(wf, O.hessian(xf), sx, 4, group, dtype=np.float32)
+    np.testing.assert_allclose(r["losses"], ref["losses"], rtol=LOSS_RTOL)
+    if r["best"] != ref["best"]:
+        a, b = ref["losses"][r["best"]], ref["losses"][ref["best"]]
+        assert abs(a - b) <= LOSS_RTOL * b, "a different alpha, not a near tie"
+    s = A.scales_for(sx, ref["alphas"][r["best"]], np.float32)
+    np.testing.assert_array_equal(r["s"], s)
+    q = A.quantize_scaled(wf, s, 4, group, np.float32)
+    _check_codes(r["codes"], q["codes"])
+    _check_codes(r["zeros"], q["zeros"])
+    same = (r["zeros"] == q["zeros"])
+    np.testing.assert_allclose(r["scales"][same], q["scales"][same], rtol=1e-6)
+    return ref
+
+
+@pytest.mark.parametrize("group", [128, 64, 32, 0])
+def test_awq_search_matches_oracle(G, group):
+    spec = synth.tiny_spec(64, 512, 2000, seed=11 + group).with_(outlier_scale=30.0)
+    x, w = synth.gen_tokens(spec), synth.gen_weight(spec)
+    r = _gpu_search(G, x, w, group)
+    ref = _check_against_oracle(r, x, w, group)
+    assert ref["best"] > 0  # the outlier channels make some alpha > 0 worth it
+
+
+def test_awq_ragged_rows_and_a_silent_channel(G):
+    spec = synth.tiny_spec(70, 256, 999, seed=5).with_(outlier_scale=20.0)
+    x, w = synth.gen_tokens(spec), synth.gen_weight(spec)
+    x[:, 17] = 0.0  # s_X = 0: the channel keeps s = 1
+    r = _gpu_search(G, x, w, 64)
+    _check_against_oracle(r, x, w, 64)
+    assert r["s"][17] == 1.0 and r["sx"][17] == 0.0
+
+
+def test_awq_larger_layer(G):
+    spec = synth.tiny_spec(512, 2048, 8192, seed=3).with_(outlier_scale=25.0)
+    x, w = synth.gen_tokens(spec), synth.gen_weight(spec)
+    r = _gpu_search(G, x, w, 128)
+    _check_against_oracle(r, x, w, 128)
+
+
+def test_awq_full_size_q_proj(G):
+    """LLaMA-7B q_proj (4096 x 4096) with 32768 calibration tokens (the AWQ
+    section's ~32K): the GPU's losses at alpha = 0 and at the chosen alpha
+    against the oracle's, and the codes at the chosen alpha."""
+    spec = synth.Q_PROJ_7B.with_(n_tokens=32768)
+    x, w = synth.gen_tokens(spec), synth.gen_weight(spec)
+    r = _gpu_search(G, x, w, 128)
+    xf = x.float().numpy()
+    wf = w.numpy().astype(np.float64)
+    sx = A.channel_scale(xf)
+    np.testing.assert_array_equal(r["sx"], sx)
+    h = O.hessian(xf)
+    alphas = A.alpha_grid()
+    for a in sorted({0, r["best"]}):
+        q = A.quantize_scaled(wf, A.scales_for(sx, alphas[a], np.float32), 4, 128, np.float32)
+        ref = O.layer_loss_hessian(wf, q["w_hat"], h)
+        assert r["losses"][a] == pytest.approx(ref, rel=LOSS_RTOL)
+    assert r["losses"][r["best"]] == r["losses"].min()
+    np.testing.assert_array_equal(r["s"], A.scales_for(sx, alphas[r["best"]], np.float32))
+    _check_codes(r["codes"], q["codes"])
