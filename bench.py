@@ -859,7 +859,10 @@ def run_awq(args, rank, world, local_rank):
         "roofline": {"bound": "tensor", "kernel": "trailing_tf32x3_kernel (dW H), over the "
                                                   "whole search stage",
                      "achieved": achieved, "peak": tf32_peak, "unit": "TFLOP/s",
-                     "frac": achieved / tf32_peak, "traffic": None,
+                     "frac": achieved / tf32_peak,
+                     "traffic": kernel_traffic("trailing_tf32x3_kernel/awq_q_proj_4096",
+                                               "post_weight_quantization_26_b200/csrc/trailing_tf32.cuh")
+                     if (dr, d) == (4096, 4096) else None,
                      "peak_source": f"bf16_tflops_sustained of {peak_src} x 1.1/2.25 "
                                     "(nominal tf32/bf16)"},
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clk,
