@@ -30,18 +30,21 @@
 //
 // Memory.  A CTA owns 16-row tiles (persistent: tile = blockIdx.x + i
 // gridDim.x); its 8 warps split each tile's columns into work items of 16
-// rows x 256 columns (warp w: items w, w + 8, ...), and a shared-memory sum
-// over the warps at the end of the tile gives Y.  Each warp streams its own
-// items through a private ring of D shared-memory slots with 16-byte
-// cp.async copies (the weights of an item, 2 KB, and its activation rows),
-// D - 1 items ahead of the one it computes, so no other warp and no
-// barrier sits on its path; 16 warps per SM keep up to 96 KB of weights in
-// flight.  The slots' row pitches make every shared-memory read below free
-// of bank conflicts: lane t of a quad holds word 4 j + t of each 128-column
-// chunk (j = 0..3), so mma pair j covers 32 consecutive columns; the
-// 32-bit weight reads of 8 rows use a pitch = 16 mod 128 bytes, the 16-byte
-// activation reads of 2 rows a pitch = 64 mod 128.  Scales and zero points
-// of the next item are loaded into registers one item ahead.
+// rows x 128 CPI columns (warp w: items w, w + 8, ...; CPI = 2 where the
+// scale regions are whole chunks and the batch is at most 4, else 1), and a
+// shared-memory sum over the warps at the end of the tile gives Y.  Each
+// warp streams its own items through a private ring of D shared-memory slots
+// with 16-byte cp.async copies (an item's weights and activation rows), D - 1
+// items ahead of the one it computes (D from 2 to 8, sized to 13.5 KB per
+// warp), so no other warp and no barrier sits on its path; at batch 1 the 16
+// warps of an SM keep 96 KB of weights in flight.  The slots' row pitches
+// make every shared-memory read below free of bank conflicts: lane t of a
+// quad holds word 4 j + t of each 128-column chunk (j = 0..3), so mma pair j
+// covers 32 consecutive columns; the weight pitch is an odd number of
+// 16-byte units (the 32-bit reads of 8 rows fall in 8 distinct groups of 4
+// banks) and the activation pitch is 4 mod 8 units (the 16-byte reads of 2
+// rows fall in distinct halves).  Scales and zero points of the next item
+// are loaded into registers one item ahead.
 #pragma once
 
 #include <cuda_bf16.h>
