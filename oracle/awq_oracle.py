@@ -1,8 +1,8 @@
 """Plain, slow, fp64 CPU oracle for the AWQ scale search.
 
 TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
-CPU-baseline legs of ``bench.py`` import this module.  It shares no code with the CUDA library,
-and the library never imports it.
+CPU-baseline legs of ``bench.py`` import this module.  It shares no code
+with the CUDA library, and the library never imports it.
 
 What it follows (dingiv.github.io "量化" page, section AWQ):
 
