@@ -11,7 +11,15 @@ on the data path).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Prints one JSON line (rank 0).
+Prints one JSON line (rank 0).  Other measurements of the same library, each
+its own JSON line:
+
+    --w4a16 BATCH    the dequant-fused 4-bit matmul over the three LLaMA-65B MLP
+                     layers (bytes streamed/s against HBM)
+    --awq            the AWQ scale search on the q_proj layer, 32768 tokens
+    --shard-layer    one q_proj layer strong-scaled across the ranks
+                     (token-sharded H + all-reduce, row-sharded quantize)
+    --bits N, --sym  other code widths / the symmetric quantizer, same path
 """
 from __future__ import annotations
 
