@@ -9,7 +9,16 @@
  * immediate in-block error updates and one lazy batched update of the columns
  * to the right after each block.  Output is b-bit codes (b = 2, 3, 4) with a
  * scale and zero point per output channel or per group of input columns
- * (granularity as on the psvmc.cn page, section 按量化粒度划分).
+ * (granularity as on the psvmc.cn page, section 按量化粒度划分).  Widths 5 to 8
+ * use the same path (section AWQ vs GPTQ names 8-bit GPTQ).
+ *
+ * Around the quantizer, the same library serves two steps the pages name:
+ *  - gptq_w4a16_matmul multiplies activations by a packed 4-bit layer
+ *    without writing the dequantized weights (section GPTQ: 4-bit weights
+ *    for memory-bound decoding);
+ *  - gptq_awq_channel_scale and gptq_awq_search run the AWQ scale search
+ *    (section AWQ) on the same calibration Hessian and produce 4-bit output
+ *    in the same format.
  *
  * Conventions for every call:
  *  - All array pointers are DEVICE pointers owned by the caller; the library
@@ -19,9 +28,10 @@
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default).
  *  - Calls validate their arguments first; on GPTQ_ERR_INVALID or
  *    GPTQ_ERR_WORKSPACE nothing is launched and no output is written.
- *  - gptq_hessian_accumulate and gptq_quantize_layer are asynchronous and do
- *    not synchronize.  gptq_prepare_hinv and gptq_dequant_check synchronize
- *    `stream` once to return a status / value.
+ *  - gptq_hessian_accumulate, gptq_quantize_layer, gptq_w4a16_matmul and the
+ *    AWQ calls are asynchronous and do not synchronize.  gptq_prepare_hinv
+ *    and gptq_dequant_check synchronize `stream` once to return a status /
+ *    value.
  *  - Kernels never spin without bound.  A kernel whose internal wait runs out
  *    records GPTQ_ERR_TIMEOUT in a device status word, frees what it holds
  *    and returns; gptq_device_status() (or the next synchronizing call)
