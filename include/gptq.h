@@ -252,7 +252,8 @@ size_t gptq_awq_workspace_size(int64_t d_row, int64_t d_col, const gptq_config* 
  *           writes it (device, 16-byte aligned, read).
  *  sx       fp64[d_col] from gptq_awq_channel_scale (device).
  *  cfg      bits 4, sym 0, group_size 0 (one scale per row) or a multiple of
- *           32 dividing d_col; d_col a multiple of 32, <= 65536.
+ *           32 dividing d_col; d_col a multiple of 32, <= 65536;
+ *           d_row * d_col < 2^31.
  *  n_grid   grid points, 2 to 64 (the AWQ section uses 20).
  *  losses   fp64[n_grid] (device, written): L(alpha_a).
  *  best     int32 (device, written): a of the best alpha.

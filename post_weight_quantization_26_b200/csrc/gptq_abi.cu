@@ -227,8 +227,10 @@ AwqWs awq_layout(int64_t d_row, int64_t d_col) {
 }
 
 bool awq_config_ok(const gptq_config* cfg, int64_t d_row, int64_t d_col) {
+  // the per-(row, group) work items are counted in int
   return config_ok(cfg, d_col) && cfg->bits == 4 && cfg->sym == 0 && d_row >= 1 &&
-         d_row <= (int64_t(1) << 24) && d_col >= 32 && d_col % 32 == 0 && d_col <= 65536;
+         d_row <= (int64_t(1) << 24) && d_col >= 32 && d_col % 32 == 0 && d_col <= 65536 &&
+         d_row * d_col <= int64_t(INT32_MAX);
 }
 
 // 2D fp32 tensor map: dims {inner, outer}, row stride in elements, box {bx, by}.

@@ -153,6 +153,7 @@ def test_awq_validation(lib):
     assert wsz(64, 256, ctypes.byref(bad3)) == 0          # AWQ is 4-bit only
     assert wsz(64, 256, ctypes.byref(sym)) == 0           # asymmetric quantizer
     assert wsz(64, 48, ctypes.byref(G.make_config(bits=4))) == 0  # d_col % 32
+    assert wsz(1 << 16, 1 << 15, ctypes.byref(g128)) == 0            # 2^31 weights
     cs = lib.gptq_awq_channel_scale
     assert cs(FAKE, 0, 64, 64, FAKE, None) == 1            # no tokens
     assert cs(FAKE, 16, 12, 16, FAKE, None) == 1           # d % 8
