@@ -29,8 +29,10 @@ Readings of points the pages leave open (each also listed in the design
 notes): the matrix norm is the squared Frobenius norm; ``G`` is the upper
 triangular ``U`` with ``U^T U = H^-1``; asymmetric codes live in
 ``[0, 2^b - 1]`` with ``s = (max(0,xmax) - min(0,xmin)) / (2^b - 1)`` and
-``z = rint(-xmin / s)``; symmetric codes use ``s = max|x| / (2^(b-1) - 1)``,
-clip to ``[-2^(b-1), 2^(b-1) - 1]`` and are stored offset by ``2^(b-1)``;
+``z = rint(-xmin / s)``, the quotient taken with s exact, i.e.
+``rint((2^b - 1) (-xmin) / (xmax - xmin))`` with one rounding; symmetric
+codes use ``s = max|x| / (2^(b-1) - 1)``, clip to ``[-2^(b-1), 2^(b-1) - 1]``
+and are stored offset by ``2^(b-1)``;
 rounding is half-to-even; group parameters come from the current (already
 error-updated) weights at the group's first column, per-channel parameters
 from the original weights; the damping adds ``damp * mean(diag H)`` to the
@@ -147,7 +149,11 @@ def quant_params(x, bits: int, sym: bool, dtype=F64):
         xmin = np.where(both0, dtype(-1), xmin)
         xmax = np.where(both0, dtype(1), xmax)
         s = (xmax - xmin) / maxq
-        z = np.rint(-xmin / s)
+        # z = rint(-xmin / s) with s = (xmax - xmin) / maxq taken exactly, as
+        # one fp64 division of (for fp32 data) exact operands.  A tie, such
+        # as a symmetric range (7.5 at 4 bits), is then rounded half to even
+        # as the formula says, instead of being decided by how s rounded.
+        z = np.rint(F64(maxq) * (-xmin.astype(F64)) / (xmax.astype(F64) - xmin.astype(F64)))
     return s.astype(dtype), z.astype(dtype)
 
 

@@ -39,6 +39,16 @@ def test_quantizer_hand_cases(case):
                                rtol=1e-15, atol=1e-15)
 
 
+@pytest.mark.parametrize("case", _load("quantizer_cases.json")["zero_tie_cases"],
+                         ids=lambda c: c["id"])
+@pytest.mark.parametrize("dtype", [np.float64, np.float32])
+def test_zero_point_ties(case, dtype):
+    """An exact tie in -xmin/s is rounded half to even, in either decision
+    precision (the quotient is formed with s exact)."""
+    _, z = O.quant_params(np.array([case["x"]]), case["bits"], False, dtype=dtype)
+    assert z[0] == case["zero"]
+
+
 @pytest.mark.parametrize("case", _load("quantizer_cases.json")["clip_cases"],
                          ids=lambda c: c["id"])
 def test_quantizer_clip(case):
