@@ -34,8 +34,8 @@
  *    value.
  *  - Kernels never spin without bound.  A kernel whose internal wait runs out
  *    records GPTQ_ERR_TIMEOUT in a device status word, frees what it holds
- *    and returns; gptq_device_status() (or the next synchronizing call)
- *    reports it.
+ *    and returns; gptq_device_status() reports it.  gptq_quantize_layer
+ *    reports a non-finite weight through the same word.
  */
 #ifndef GPTQ_B200_H
 #define GPTQ_B200_H
@@ -51,7 +51,7 @@ typedef enum {
   GPTQ_OK = 0,
   GPTQ_ERR_INVALID = 1,    /* bad argument: null pointer, size, alignment, config */
   GPTQ_ERR_NOT_SPD = 2,    /* damped H is not positive definite (see bad_pivot) */
-  GPTQ_ERR_NONFINITE = 3,  /* NaN or Inf found in H (prepare) */
+  GPTQ_ERR_NONFINITE = 3,  /* NaN or Inf found in H (prepare) or in W (quantize) */
   GPTQ_ERR_WORKSPACE = 4,  /* workspace null, misaligned or smaller than required */
   GPTQ_ERR_CUDA = 5,       /* a CUDA runtime call or launch failed */
   GPTQ_ERR_TIMEOUT = 6     /* a kernel's bounded internal wait ran out */
@@ -68,7 +68,9 @@ typedef enum {
  *              reached.  Must be a multiple of 32 that divides d_col, with
  *              block % group_size == 0 or group_size % block == 0.
  *  sym         0: asymmetric, codes q = clip(rint(w/s) + z, 0, 2^b-1) with
- *                 s = (max(0,max w) - min(0,min w)) / (2^b-1), z = rint(-min(0,min w)/s);
+ *                 s = (max(0,max w) - min(0,min w)) / (2^b-1), z = rint(-min(0,min w)/s)
+ *                 where the quotient is formed with s exact (one fp64
+ *                 division), so an exact tie rounds half to even;
  *              1: symmetric, s = max|w| / (2^(b-1)-1), z = 2^(b-1) (codes
  *                 stored offset-binary, i.e. signed code + 2^(b-1)).
  *              Dequantized value: s * (q - z).  (dingiv.github.io page,
@@ -99,14 +101,29 @@ size_t gptq_workspace_size(int64_t d_row, int64_t d_col, const gptq_config* cfg)
  *         elements (ldx >= d, ldx % 8 == 0, X 16-byte aligned).  This is
  *         X^T of the page's d x n matrix, the layout a model's activations
  *         have.  Chunks of any size may be accumulated by repeated calls.
- *  d      % 8 == 0, 8 <= d <= 65536.   n >= 0 (n == 0 is a no-op and X may
- *         then be NULL).
- * Summation order over tokens within one call is not fixed (split over
- * tokens with fp32 atomic adds), so results may differ in the last bits
- * between runs.  Asynchronous. */
+ *  d      % 8 == 0, 8 <= d <= 65536.   0 <= n < 2^31 - 64 (n == 0 is a
+ *         no-op and X may then be NULL).
+ * Each 128 x 256 tile of H sums its tokens on the tensor cores (fp32
+ * accumulation, restarted every 1024 tokens and folded with round-to-nearest
+ * adds).  When the tiles are too few to fill the GPU, the tokens are split
+ * into chunks whose partial sums meet in H through TMA reduce-adds in L2,
+ * in an order that varies between runs, so H may then differ in the last
+ * bits from run to run (gptq_hessian_accumulate_ordered fixes the order).
+ * Asynchronous. */
 gptq_status gptq_hessian_accumulate(float* H, const void* X, int64_t n,
                                     int64_t d, int64_t ldx, float scale,
                                     void* stream);
+
+/* gptq_hessian_accumulate with a fixed summation order: the tokens of a call
+ * are never split, so every element of H receives exactly one add per call
+ * and, for the same H, X and chunking, H is bitwise reproducible.  Same
+ * arguments and errors.  It costs up to about 10% of the Hessian stage where
+ * the tile count leaves the last wave of SMs part-empty (d = 4096: 272 tiles
+ * on 148 SMs) and nothing where the tiles fill the GPU anyway (d >= 11008).
+ * Asynchronous. */
+gptq_status gptq_hessian_accumulate_ordered(float* H, const void* X, int64_t n,
+                                            int64_t d, int64_t ldx, float scale,
+                                            void* stream);
 
 /* From H (upper triangle, as left by gptq_hessian_accumulate) compute the
  * damped H' = H + lambda I, lambda = damp_rel * mean(diag H), with a dead
@@ -145,7 +162,10 @@ gptq_status gptq_prepare_hinv(const float* H, int64_t d, double damp_rel,
  *  scales     fp32 d_row x n_groups output (n_groups = 1 when group_size is
  *             0, else d_col / group_size), row-major.
  *  zeros      uint8 d_row x n_groups output (integer zero points).
- *  Shapes: d_row >= 1, d_col % 32 == 0, d_col >= 32.  Asynchronous. */
+ *  Shapes: d_row >= 1, d_col % 32 == 0, d_col >= 32.  Asynchronous.
+ * A NaN or Inf in W (outside dead columns) sets the device status word to
+ * GPTQ_ERR_NONFINITE, reported by the next gptq_device_status(); the outputs
+ * of that call are then meaningless. */
 gptq_status gptq_quantize_layer(const float* W, int64_t d_row, int64_t d_col,
                                 const float* G, const uint8_t* dead_mask,
                                 const gptq_config* cfg, uint32_t* qweight,
@@ -188,8 +208,10 @@ gptq_status gptq_dequant_check(const uint32_t* qweight, const float* scales,
  *  Layers with more tiles than GPTQ_NOALLOC_MAX_TILES are rejected with
  *  GPTQ_ERR_INVALID (and a message on stderr) before anything is launched.
  *  The first call on a device looks up that array's device address (once per
- *  device, with that device current); make that first call before any
- *  stream capture.
+ *  device and CUDA context, with that device current); make that first call
+ *  before any stream capture.  After a device reset (cudaDeviceReset, or a
+ *  framework that resets the device) the new context holds a new copy of the
+ *  array, and the next call looks its address up again.
  *  All calls share the one array, which keeps the last call's contents; each
  *  call overwrites every entry it later reads, so nothing needs clearing, but
  *  calls that overlap on the GPU (other streams, other host threads) race on
@@ -272,8 +294,28 @@ gptq_status gptq_awq_search(const float* W, const float* H, const double* sx, in
                             uint8_t* zeros, void* ws, size_t ws_bytes, void* stream);
 
 /* Synchronize `stream`, then return and clear the device status word that
- * kernels set when a bounded internal wait runs out (GPTQ_ERR_TIMEOUT). */
+ * kernels set when a bounded internal wait runs out (GPTQ_ERR_TIMEOUT) or
+ * when gptq_quantize_layer meets a non-finite weight (GPTQ_ERR_NONFINITE).
+ * The first such event since the last call is kept. */
 gptq_status gptq_device_status(void* stream);
+
+/* Fault injection for testing the failure detection; the paper has no
+ * counterpart.  Off (GPTQ_FAULT_NONE) unless set, process-wide, and applied
+ * to every later launch until changed:
+ *  where          GPTQ_FAULT_SYRK_STALL: the producer warp of the Hessian
+ *                 kernel issues no loads, so the MMA thread's first bounded
+ *                 wait runs out; GPTQ_FAULT_TRAILING_STALL: the same in the
+ *                 trailing-update kernel of gptq_quantize_layer and
+ *                 gptq_awq_search.  Nothing is in flight when the waits give
+ *                 up; the kernel records GPTQ_ERR_TIMEOUT, frees its tensor
+ *                 memory and returns, and the context stays usable.  The
+ *                 outputs of a stalled call are meaningless.
+ *  wait_limit_ns  the limit of every bounded wait in every kernel, 1 ms to
+ *                 10 s; 0 restores the default of 2 s.
+ * Returns GPTQ_ERR_INVALID for other values (nothing changes then).  Not
+ * thread-safe against launches in flight on other host threads. */
+enum { GPTQ_FAULT_NONE = 0, GPTQ_FAULT_SYRK_STALL = 1, GPTQ_FAULT_TRAILING_STALL = 2 };
+gptq_status gptq_fault_inject(int where, int64_t wait_limit_ns);
 
 /* Number of kernels this library has launched in this process (all devices,
  * all streams).  Instrumentation for benchmarks: the difference across a

@@ -8,13 +8,16 @@
 
 namespace gptq {
 
-// Status word written by kernels whose bounded waits run out (0 = fine).
-// Read and cleared by the host through gptq_device_status().
+// Status word written by kernels whose bounded waits run out, or that meet a
+// non-finite weight (0 = fine).  Read and cleared by the host through
+// gptq_device_status().
 __device__ int g_device_status = 0;
 
-// A wait longer than this (ns of %globaltimer) is treated as a hang.
+// A wait longer than this (ns of %globaltimer) is treated as a hang.  The
+// kernels take the limit as a launch parameter; this is its default.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
-constexpr int kStatusTimeout = 6;  // == GPTQ_ERR_TIMEOUT
+constexpr int kStatusTimeout = 6;    // == GPTQ_ERR_TIMEOUT
+constexpr int kStatusNonfinite = 3;  // == GPTQ_ERR_NONFINITE
 
 __device__ __forceinline__ uint64_t global_timer_ns() {
   uint64_t t;
@@ -24,6 +27,10 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 
 __device__ __forceinline__ void report_timeout() {
   atomicCAS(&g_device_status, 0, kStatusTimeout);
+}
+
+__device__ __forceinline__ void report_nonfinite() {
+  atomicCAS(&g_device_status, 0, kStatusNonfinite);
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -63,17 +70,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait until the phase with the given parity has completed.  Gives up (and
-// raises the CTA's abort flag and the device status word) after
-// kWaitLimitNs, or as soon as another role of the CTA has aborted.
+// raises the CTA's abort flag and the device status word) after limit_ns of
+// %globaltimer, or as soon as another role of the CTA has aborted.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
-                                                  volatile int* abort_flag) {
+                                                  volatile int* abort_flag,
+                                                  uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 31u) == 0) {
       if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         report_timeout();
         return false;

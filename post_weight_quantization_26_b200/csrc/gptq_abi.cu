@@ -45,6 +45,11 @@ inline bool aligned(const void* p, size_t a) {
 
 std::atomic<uint64_t> g_launches{0};
 
+// Fault injection for the failure-detection tests (gptq_fault_inject): which
+// kernel's producer stalls, and the limit of every bounded wait.
+std::atomic<int> g_fault{GPTQ_FAULT_NONE};
+std::atomic<uint64_t> g_wait_ns{gptq::kWaitLimitNs};
+
 #define GPTQ_LAUNCH_CHECK()                          \
   do {                                               \
     g_launches.fetch_add(1, std::memory_order_relaxed); \
@@ -449,6 +454,8 @@ gptq_status gptq_awq_search(const float* W, const float* H, const double* sx, in
     return st;
   trail::Params tp{};
   tp.M = dr; tp.N = dc; tp.K = dc; tp.n0 = 0; tp.j0 = 0;
+  tp.wait_ns = g_wait_ns.load();
+  tp.stall = g_fault.load() == GPTQ_FAULT_TRAILING_STALL;
   tp.tiles_m = (dr + trail::BM - 1) / trail::BM;
   tp.tiles_n = (dc + trail::BN - 1) / trail::BN;
   tp.tiles = tp.tiles_m * tp.tiles_n;
@@ -489,11 +496,16 @@ gptq_status gptq_device_status(void* stream) {
   return static_cast<gptq_status>(v);
 }
 
-gptq_status gptq_hessian_accumulate(float* H, const void* X, int64_t n, int64_t d, int64_t ldx,
-                                    float scale, void* stream) {
+}  // extern "C"
+
+namespace {
+
+gptq_status hessian_accumulate(float* H, const void* X, int64_t n, int64_t d, int64_t ldx,
+                               float scale, bool ordered, void* stream) {
   if (!H) return GPTQ_ERR_INVALID;
   if (d < 8 || d > 65536 || d % 8 != 0) return GPTQ_ERR_INVALID;
-  if (n < 0 || n > (int64_t(1) << 31) - 1) return GPTQ_ERR_INVALID;
+  // token offsets and a chunk's length rounded up to BK stay below 2^31
+  if (n < 0 || n > (int64_t(1) << 31) - 1 - syrk::BK) return GPTQ_ERR_INVALID;
   if (ldx < d || ldx % 8 != 0) return GPTQ_ERR_INVALID;
   if (!std::isfinite(scale) || !aligned(H, 16)) return GPTQ_ERR_INVALID;
   if (n == 0) return GPTQ_OK;  // X may be NULL for an empty chunk
@@ -531,12 +543,44 @@ gptq_status gptq_hessian_accumulate(float* H, const void* X, int64_t n, int64_t 
     const int h = p.nti >> 1;
     p.ntiles = p.nti * p.ntj - (h * (h - 1) + (p.nti & 1) * h);
   }
-  choose_split(p.ntiles, p.n, num_sms, &p.split_tokens, &p.nsplit);
+  if (ordered) {  // one chunk: each element of H gets exactly one add
+    p.split_tokens = (p.n + syrk::BK - 1) / syrk::BK * syrk::BK;
+    p.nsplit = 1;
+  } else {
+    choose_split(p.ntiles, p.n, num_sms, &p.split_tokens, &p.nsplit);
+  }
   p.units = p.ntiles * p.nsplit;
+  p.wait_ns = g_wait_ns.load();
+  p.stall = g_fault.load() == GPTQ_FAULT_SYRK_STALL;
   const int grid = std::min(p.units, num_sms);
   syrk::syrk_bf16_tcgen05_kernel<<<grid, syrk::NUM_THREADS, syrk::SMEM_BYTES,
                                    static_cast<cudaStream_t>(stream)>>>(tmap, tmap_h, p);
   GPTQ_LAUNCH_CHECK();
+  return GPTQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+gptq_status gptq_hessian_accumulate(float* H, const void* X, int64_t n, int64_t d, int64_t ldx,
+                                    float scale, void* stream) {
+  return hessian_accumulate(H, X, n, d, ldx, scale, false, stream);
+}
+
+gptq_status gptq_hessian_accumulate_ordered(float* H, const void* X, int64_t n, int64_t d,
+                                            int64_t ldx, float scale, void* stream) {
+  return hessian_accumulate(H, X, n, d, ldx, scale, true, stream);
+}
+
+gptq_status gptq_fault_inject(int where, int64_t wait_limit_ns) {
+  if (where != GPTQ_FAULT_NONE && where != GPTQ_FAULT_SYRK_STALL &&
+      where != GPTQ_FAULT_TRAILING_STALL)
+    return GPTQ_ERR_INVALID;
+  if (wait_limit_ns != 0 && (wait_limit_ns < 1000000 || wait_limit_ns > 10000000000ll))
+    return GPTQ_ERR_INVALID;
+  g_wait_ns.store(wait_limit_ns ? static_cast<uint64_t>(wait_limit_ns) : gptq::kWaitLimitNs);
+  g_fault.store(where);
   return GPTQ_OK;
 }
 
@@ -767,6 +811,8 @@ gptq_status gptq_quantize_layer(const float* W, int64_t d_row, int64_t d_col, co
       GPTQ_CUDA_TRY(cudaStreamWaitEvent(di->aux, evQ[jb % 4], 0));
       trail::Params tp{};
       tp.M = dr; tp.N = dc - n0; tp.K = ncols; tp.n0 = n0; tp.j0 = j0;
+      tp.wait_ns = g_wait_ns.load();
+      tp.stall = g_fault.load() == GPTQ_FAULT_TRAILING_STALL;
       tp.tiles_m = (dr + trail::BM - 1) / trail::BM;
       tp.tiles_n = (tp.N + trail::BN - 1) / trail::BN;
       tp.tiles = tp.tiles_m * tp.tiles_n;
@@ -834,14 +880,31 @@ static __device__ __align__(256) double g_noalloc_scratch[GPTQ_NOALLOC_MAX_TILES
 
 namespace {
 std::mutex g_noalloc_mu;
+// Per device: the array's device address and the context it was looked up
+// in.  A device reset (cudaDeviceReset, or a framework that resets the
+// device) makes a new primary context with a new copy of the array, so the
+// address is looked up again whenever the current context differs.
 double* g_noalloc_ptr[64] = {};
+CUcontext g_noalloc_ctx[64] = {};
+PFN_cuCtxGetCurrent_v4000 g_ctx_current = nullptr;
 
 gptq_status noalloc_scratch(double** out) {
   int dev = 0;
   GPTQ_CUDA_TRY(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64) return GPTQ_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  if (!g_ctx_current) {
+    cudaDriverEntryPointQueryResult q;
+    void* fn = nullptr;
+    GPTQ_CUDA_TRY(cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q));
+    if (q != cudaDriverEntryPointSuccess || !fn) return GPTQ_ERR_CUDA;
+    g_ctx_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(fn);
+  }
+  // No context current on this thread yet (or another one): look the
+  // address up, which also makes the device's primary context current.
+  CUcontext ctx = nullptr;
+  if (g_ctx_current(&ctx) != CUDA_SUCCESS) return GPTQ_ERR_CUDA;
+  if (!ctx || !g_noalloc_ptr[dev] || g_noalloc_ctx[dev] != ctx) {
     void* p = nullptr;
     cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || !p) {
@@ -849,7 +912,9 @@ gptq_status noalloc_scratch(double** out) {
                    cudaGetErrorString(e));
       return GPTQ_ERR_CUDA;
     }
+    if (g_ctx_current(&ctx) != CUDA_SUCCESS || !ctx) return GPTQ_ERR_CUDA;
     g_noalloc_ptr[dev] = static_cast<double*>(p);
+    g_noalloc_ctx[dev] = ctx;
   }
   *out = g_noalloc_ptr[dev];
   return GPTQ_OK;

@@ -21,8 +21,9 @@
 // sections 二 and 四): asymmetric q = clip(rint(w/s) + z, 0, 2^b-1) with
 // s = (max(0,max) - min(0,min)) / (2^b-1), z = rint(-min(0,min)/s);
 // symmetric s = max|w| / (2^(b-1)-1), z = 2^(b-1); w^ = s (q - z).  The
-// integer decisions are taken in fp32 with IEEE division and
-// round-half-to-even.
+// codes are decided in fp32 with IEEE division and round-half-to-even; the
+// zero point is rint((2^b-1)(-min)/(max-min)) as one fp64 division of exact
+// operands, which is -min/s with s unrounded.
 #pragma once
 
 #include "common.cuh"
@@ -41,13 +42,20 @@ __device__ __forceinline__ void make_params(float mn, float mx, int bits, int sy
     mn = fminf(mn, 0.0f);
     mx = fmaxf(mx, 0.0f);
     if (mn == 0.0f && mx == 0.0f) { mn = -1.0f; mx = 1.0f; }
-    s = (mx - mn) / static_cast<float>((1 << bits) - 1);
-    z = rintf(-mn / s);
+    const int maxq = (1 << bits) - 1;
+    s = (mx - mn) / static_cast<float>(maxq);
+    // z = rint(-mn / s) with s taken exactly: one fp64 division of exact
+    // operands, so an exact tie (a symmetric range gives 7.5 at 4 bits) is
+    // rounded half to even rather than decided by the rounding of s.
+    z = static_cast<float>(rint(static_cast<double>(maxq) * static_cast<double>(-mn) /
+                                (static_cast<double>(mx) - static_cast<double>(mn))));
   }
 }
 
 // Copy W into the working buffer (dead columns zeroed) and, for one scale per
-// output channel, compute each row's parameters from that copy.  One warp per row.
+// output channel, compute each row's parameters from that copy.  One warp per
+// row.  A NaN or Inf outside the dead columns sets the device status word to
+// GPTQ_ERR_NONFINITE.
 __global__ void prepare_rows_kernel(const float* __restrict__ W, float* __restrict__ Wk,
                                     const uint8_t* __restrict__ dead, int d_row, int d_col,
                                     int bits, int sym, int per_channel,
@@ -58,6 +66,7 @@ __global__ void prepare_rows_kernel(const float* __restrict__ W, float* __restri
   const float4* src = reinterpret_cast<const float4*>(W + static_cast<size_t>(r) * d_col);
   float4* dst = reinterpret_cast<float4*>(Wk + static_cast<size_t>(r) * d_col);
   float mn = 0.0f, mx = 0.0f;
+  bool finite = true;
   for (int c4 = lane; c4 < d_col / 4; c4 += 32) {
     float4 v = src[c4];
     if (dead) {
@@ -68,9 +77,11 @@ __global__ void prepare_rows_kernel(const float* __restrict__ W, float* __restri
       if (dm.w) v.w = 0.0f;
     }
     dst[c4] = v;
+    finite = finite && isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w);
     mn = fminf(mn, fminf(fminf(v.x, v.y), fminf(v.z, v.w)));
     mx = fmaxf(mx, fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
   }
+  if (!__all_sync(0xffffffffu, finite) && lane == 0) report_nonfinite();
   if (!per_channel) return;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {

@@ -13,7 +13,9 @@
 // relative after 2300 MMAs, measured against an fp64 sum).  So a TMEM
 // accumulator only ever sums CHAIN_TOKENS tokens from zero; each finished
 // chain is folded into fp32 registers of the epilogue with ordinary
-// round-to-nearest adds, and the chunk's sum leaves through the atomics.
+// round-to-nearest adds, and the chunk's sum leaves through a TMA reduce-add.
+// With one chunk (nsplit = 1) every element of H receives exactly one add
+// per launch, so H does not depend on the order in which units finish.
 //
 // Warp roles (320 threads, one CTA per SM, persistent over work units):
 //   warp 0      TMA producer: 64-token stages, A = 2 boxes of 64 features,
@@ -71,6 +73,9 @@ struct Params {
   int split_tokens;  // tokens per chunk (multiple of BK)
   int nsplit;
   int units;      // ntiles * nsplit
+  uint64_t wait_ns;  // limit of every bounded wait (ns)
+  int stall;      // fault injection: the producer issues nothing, so the
+                  // MMA thread's first wait runs out (0 in normal use)
 };
 
 // Tiles of row-tile ti that touch the upper triangle start at column tile
@@ -143,14 +148,14 @@ syrk_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_x,
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    if (lane == 0 && !p.stall) {
       uint32_t stage = 0, phase = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
         int ti, tj, k0, nk;
         decode_unit(p, u, ti, tj, k0, nk);
         for (int kt = 0; kt < nk; ++kt) {
-          if (!mbar_wait_bounded(empty0 + 8u * stage, phase ^ 1u, abort_flag)) { ok = false; break; }
+          if (!mbar_wait_bounded(empty0 + 8u * stage, phase ^ 1u, abort_flag, p.wait_ns)) { ok = false; break; }
           const uint32_t fb = full0 + 8u * stage;
           mbar_arrive_expect_tx(fb, STAGE_BYTES);
           const uint32_t sa = ring + stage * STAGE_BYTES;
@@ -178,11 +183,11 @@ syrk_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_x,
           const int kc = kt % CHAIN_KB;
           if (kc == 0) {  // a new chain starts in the other accumulator
             const uint32_t acc = gc & 1u;
-            if (!mbar_wait_bounded(tempty0 + 8u * acc, ((gc >> 1) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+            if (!mbar_wait_bounded(tempty0 + 8u * acc, ((gc >> 1) & 1u) ^ 1u, abort_flag, p.wait_ns)) { ok = false; break; }
             tc_fence_after();
             d_tmem = tmem_base + acc * BN;
           }
-          if (!mbar_wait_bounded(full0 + 8u * stage, phase, abort_flag)) { ok = false; break; }
+          if (!mbar_wait_bounded(full0 + 8u * stage, phase, abort_flag, p.wait_ns)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = ring + stage * STAGE_BYTES;
           const uint32_t sb = sa + A_BYTES;
@@ -221,7 +226,7 @@ syrk_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_x,
       const int nchains = (nk + CHAIN_KB - 1) / CHAIN_KB;
       for (int ch = 0; ch < nchains; ++ch, ++gc) {
         const uint32_t acc = gc & 1u;
-        if (ok && !mbar_wait_bounded(tfull0 + 8u * acc, (gc >> 1) & 1u, abort_flag)) ok = false;
+        if (ok && !mbar_wait_bounded(tfull0 + 8u * acc, (gc >> 1) & 1u, abort_flag, p.wait_ns)) ok = false;
         if (!ok) continue;
         tc_fence_after();
         const uint32_t t0 = tmem_base + lane_off + acc * BN + half * (BN / 2);

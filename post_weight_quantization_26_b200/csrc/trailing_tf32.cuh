@@ -58,6 +58,9 @@ struct Params {
   int n0;       // first column to update (also the column coordinate into G)
   int j0;       // first row of G's block
   int tiles_m, tiles_n, tiles;
+  uint64_t wait_ns;  // limit of every bounded wait (ns)
+  int stall;    // fault injection: the producer issues nothing, so the MMA
+                // thread's first wait runs out (0 in normal use)
 };
 
 __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo,
@@ -124,13 +127,13 @@ trailing_tf32x3_kernel(const __grid_constant__ CUtensorMap tm_ehi,
   const int nk = (p.K + BK - 1) / BK;  // E is zero past K
 
   if (warp == 0) {
-    if (lane == 0) {  // ------------------------------------------- producer
+    if (lane == 0 && !p.stall) {  // -------------------------------- producer
       uint32_t stage = 0, phase = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < p.tiles && ok; u += gridDim.x) {
         const int tm = u % p.tiles_m, tn = u / p.tiles_m;
         for (int ks = 0; ks < nk; ++ks) {
-          if (!mbar_wait_bounded(empty0 + 8u * stage, phase ^ 1u, abort_flag)) { ok = false; break; }
+          if (!mbar_wait_bounded(empty0 + 8u * stage, phase ^ 1u, abort_flag, p.wait_ns)) { ok = false; break; }
           const uint32_t fb = full0 + 8u * stage;
           mbar_arrive_expect_tx(fb, STAGE_BYTES);
           const uint32_t s0 = ring + stage * STAGE_BYTES;
@@ -154,11 +157,11 @@ trailing_tf32x3_kernel(const __grid_constant__ CUtensorMap tm_ehi,
       bool ok = true;
       for (int u = blockIdx.x; u < p.tiles && ok; u += gridDim.x, ++lu) {
         const uint32_t acc = lu & 1;
-        if (!mbar_wait_bounded(tempty0 + 8u * acc, ((lu >> 1) & 1) ^ 1u, abort_flag)) break;
+        if (!mbar_wait_bounded(tempty0 + 8u * acc, ((lu >> 1) & 1) ^ 1u, abort_flag, p.wait_ns)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int ks = 0; ks < nk; ++ks) {
-          if (!mbar_wait_bounded(full0 + 8u * stage, phase, abort_flag)) { ok = false; break; }
+          if (!mbar_wait_bounded(full0 + 8u * stage, phase, abort_flag, p.wait_ns)) { ok = false; break; }
           tc_fence_after();
           const uint32_t s0 = ring + stage * STAGE_BYTES;
 #pragma unroll
@@ -197,7 +200,7 @@ trailing_tf32x3_kernel(const __grid_constant__ CUtensorMap tm_ehi,
     for (int u = blockIdx.x; u < p.tiles; u += gridDim.x, ++lu) {
       const int tm = u % p.tiles_m, tn = u / p.tiles_m;
       const uint32_t acc = lu & 1;
-      if (ok && !mbar_wait_bounded(tfull0 + 8u * acc, (lu >> 1) & 1, abort_flag)) ok = false;
+      if (ok && !mbar_wait_bounded(tfull0 + 8u * acc, (lu >> 1) & 1, abort_flag, p.wait_ns)) ok = false;
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
       for (int c = 0; c < BN / OUT_COLS; ++c) {

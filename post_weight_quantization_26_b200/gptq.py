@@ -23,11 +23,12 @@ STATUS_NAMES = {0: "GPTQ_OK", 1: "GPTQ_ERR_INVALID", 2: "GPTQ_ERR_NOT_SPD",
                 5: "GPTQ_ERR_CUDA", 6: "GPTQ_ERR_TIMEOUT"}
 
 EXPORTED = ("gptq_workspace_size", "gptq_hessian_accumulate",
-            "gptq_prepare_hinv", "gptq_quantize_layer", "gptq_dequant_check",
+            "gptq_hessian_accumulate_ordered", "gptq_fault_inject", "gptq_prepare_hinv", "gptq_quantize_layer", "gptq_dequant_check",
             "gptq_device_status", "gptq_status_string", "gptq_launch_count",
             "gptq_dequant_check_noalloc", "gptq_w4a16_matmul", "gptq_awq_channel_scale",
             "gptq_awq_workspace_size", "gptq_awq_search")
 NOALLOC_MAX_TILES = 65536  # GPTQ_NOALLOC_MAX_TILES in include/gptq.h
+FAULT_NONE, FAULT_SYRK_STALL, FAULT_TRAILING_STALL = 0, 1, 2  # GPTQ_FAULT_* in include/gptq.h
 
 
 class GptqError(RuntimeError):
@@ -67,6 +68,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gptq_workspace_size.restype = SZ
     lib.gptq_hessian_accumulate.argtypes = [P, P, I64, I64, I64, F, P]
     lib.gptq_hessian_accumulate.restype = I
+    lib.gptq_hessian_accumulate_ordered.argtypes = [P, P, I64, I64, I64, F, P]
+    lib.gptq_hessian_accumulate_ordered.restype = I
+    lib.gptq_fault_inject.argtypes = [I, I64]
+    lib.gptq_fault_inject.restype = I
     lib.gptq_prepare_hinv.argtypes = [P, I64, D, P, P, P, SZ,
                                       ctypes.POINTER(I64), P]
     lib.gptq_prepare_hinv.restype = I
@@ -132,12 +137,30 @@ def alloc_workspace(d_row: int, d_col: int, cfg: GptqConfig, device=None):
 def gptq_hessian_accumulate(H: torch.Tensor, X: torch.Tensor,
                             scale: float = 2.0, stream=None) -> None:
     """H (fp32 d x d) += scale * X^T X for token-major bf16 X (n x d)."""
+    _accumulate("gptq_hessian_accumulate", H, X, scale, stream)
+
+
+def gptq_hessian_accumulate_ordered(H: torch.Tensor, X: torch.Tensor,
+                                    scale: float = 2.0, stream=None) -> None:
+    """gptq_hessian_accumulate with a fixed summation order (bitwise
+    reproducible H)."""
+    _accumulate("gptq_hessian_accumulate_ordered", H, X, scale, stream)
+
+
+def _accumulate(name, H, X, scale, stream):
     assert H.dtype == torch.float32 and X.dtype == torch.bfloat16
     n, d = X.shape
     assert H.shape == (d, d) and H.is_contiguous() and X.stride(1) == 1
-    st = load_library().gptq_hessian_accumulate(
+    st = getattr(load_library(), name)(
         _ptr(H), _ptr(X), n, d, X.stride(0), float(scale), _stream(stream))
-    _check(st, "gptq_hessian_accumulate")
+    _check(st, name)
+
+
+def gptq_fault_inject(where: int, wait_limit_ns: int = 0) -> None:
+    """Set the fault injection of the failure-detection tests (FAULT_NONE
+    and 0 restore normal operation)."""
+    _check(load_library().gptq_fault_inject(int(where), int(wait_limit_ns)),
+           "gptq_fault_inject")
 
 
 def gptq_prepare_hinv(H: torch.Tensor, damp_rel: float, G: torch.Tensor,

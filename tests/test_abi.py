@@ -77,8 +77,9 @@ def test_workspace_size_rules(lib):
     assert lib.gptq_workspace_size(64, 384, ctypes.byref(g256)) == 0  # group must divide
 
 
-def test_hessian_accumulate_validation(lib):
-    f = lib.gptq_hessian_accumulate
+@pytest.mark.parametrize("name", ["gptq_hessian_accumulate", "gptq_hessian_accumulate_ordered"])
+def test_hessian_accumulate_validation(lib, name):
+    f = getattr(lib, name)
     assert f(None, FAKE, 16, 64, 64, 2.0, None) == 1
     assert f(FAKE, None, 16, 64, 64, 2.0, None) == 1
     assert f(FAKE, None, 0, 64, 64, 2.0, None) == 0    # empty chunk, no data
@@ -89,6 +90,19 @@ def test_hessian_accumulate_validation(lib):
     assert f(FAKE, FAKE, 16, 64, 64, float("nan"), None) == 1
     assert f(FAKE, ctypes.c_void_p(0x7F0000000002), 16, 64, 64, 2.0, None) == 1  # alignment
     assert f(FAKE, FAKE, 0, 64, 64, 2.0, None) == 0    # n == 0 is a no-op
+    assert f(FAKE, FAKE, (1 << 31) - 64, 64, 64, 2.0, None) == 1  # a chunk past 2^31 tokens
+
+
+def test_fault_inject_validation(lib):
+    """Only the documented switches and limits are accepted; normal
+    operation is restored by (NONE, 0)."""
+    from post_weight_quantization_26_b200 import gptq as G
+    f = lib.gptq_fault_inject
+    assert f(3, 0) == 1 and f(-1, 0) == 1                 # unknown switch
+    assert f(G.FAULT_SYRK_STALL, 999_999) == 1            # limit below 1 ms
+    assert f(G.FAULT_SYRK_STALL, 10_000_000_001) == 1     # limit above 10 s
+    assert f(G.FAULT_TRAILING_STALL, 20_000_000) == 0
+    assert f(G.FAULT_NONE, 0) == 0
 
 
 def test_prepare_and_quantize_validation(lib):

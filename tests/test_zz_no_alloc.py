@@ -40,10 +40,11 @@ def _quantized_layer(G, spec):
     return cfg, w, h, qw, sc, ze, ws
 
 
-@pytest.mark.parametrize("shape", [(256, 256, 0), (200, 384, 128)])
+@pytest.mark.parametrize("shape", [(256, 256, 0, 4), (200, 384, 128, 4), (192, 512, 128, 3),
+                                   (130, 256, 0, 8)])
 def test_noalloc_matches_workspace_version_twice(G, shape):
-    d_row, d_col, group = shape
-    spec = synth.tiny_spec(d_row, d_col, 1024, seed=d_row).with_(group=group)
+    d_row, d_col, group, bits = shape
+    spec = synth.tiny_spec(d_row, d_col, 1024, seed=d_row).with_(group=group, bits=bits)
     cfg, w, h, qw, sc, ze, ws = _quantized_layer(G, spec)
     w_hat_ref = torch.empty_like(w)
     loss_ref = G.gptq_dequant_check(qw, sc, ze, w, h, cfg, W_hat=w_hat_ref, ws=ws)
@@ -67,6 +68,32 @@ def test_noalloc_after_a_larger_call(G):
     ref = G.gptq_dequant_check(qw_s, sc_s, ze_s, w_s, h_s, cfg_s, ws=ws_s)
     got = G.gptq_dequant_check_noalloc(qw_s, sc_s, ze_s, w_s, h_s, cfg_s)
     assert got == pytest.approx(ref, rel=1e-12)
+
+
+def test_noalloc_many_tiles(G):
+    """A 16384 x 4096 layer: 4096 tiles of 128 x 128, so the scratch holds
+    thousands of partial sums; twice in a row, against the workspace
+    version.  The packed layer is a seeded random one in the quantizer's
+    format (only the format matters to the check)."""
+    d_row, d_col = 16384, 4096
+    words, scales, zeros = synth.gen_packed_layer(d_row, d_col, 128, seed=9)
+    cfg = G.make_config(bits=4, group_size=128)
+    spec = synth.tiny_spec(d_row, d_col, 8192, seed=9)
+    w = synth.gen_weight(spec).cuda()
+    x = synth.gen_tokens(spec).cuda()
+    h = torch.zeros((d_col, d_col), dtype=torch.float32, device="cuda")
+    G.gptq_hessian_accumulate(h, x)
+    qw, sc, ze = words.cuda(), scales.cuda(), zeros.cuda()
+    ws = G.alloc_workspace(d_row, d_col, cfg)
+    w_hat_ref = torch.empty_like(w)
+    loss_ref = G.gptq_dequant_check(qw, sc, ze, w, h, cfg, W_hat=w_hat_ref, ws=ws)
+    assert np.isfinite(loss_ref) and loss_ref > 0
+    for _ in range(2):
+        w_hat = torch.full_like(w, float("nan"))
+        loss = G.gptq_dequant_check_noalloc(qw, sc, ze, w, h, cfg, W_hat=w_hat)
+        assert loss == pytest.approx(loss_ref, rel=1e-12)
+        torch.testing.assert_close(w_hat, w_hat_ref, rtol=0, atol=0)
+    assert G.gptq_device_status() == 0
 
 
 def test_noalloc_rejects_layers_beyond_its_scratch(G):
