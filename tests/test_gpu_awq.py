@@ -2,18 +2,19 @@
 oracle on the same seeded layers and calibration tokens.
 
 Bars: the channel scale is exact (fp64 sums of bf16 magnitudes); s* equals
-the oracle's s rounded to fp32; the codes and zero points of W diag(s*) are
-those of the oracle taking its decisions in fp32 (at most 0.1% of codes off
-by one, as for the GPTQ path); each alpha's loss is within 1e-4 relative of
-the oracle's.  The loss goes through the fp32 SYRK (H relative error ~1e-7)
-and a split-TF32 contraction (~1e-6 of the product), so 1e-4 leaves room.
-The chosen alpha is the oracle's, unless the two losses involved are within
-that same tolerance of each other.
+the oracle's fp64 s rounded to fp32 storage; the codes and zero points of
+W diag(s*) are those of the fp64 oracle (at most 0.1% of codes off by one,
+as for the GPTQ path) and the scales within 1e-5; each alpha's loss is
+within 1e-4 relative of the oracle's.  The loss goes through the fp32 SYRK
+(H relative error ~1e-7) and a split-TF32 contraction (~1e-6 of the
+product), so 1e-4 leaves room.  The chosen alpha is the oracle's, unless the
+two losses involved are within that same tolerance of each other.
 """
 import numpy as np
 import pytest
 import torch
 
+from gptq_parity import check_layer
 from oracle import awq_oracle as A
 from oracle import gptq_oracle as O
 from post_weight_quantization_26_b200 import synth
@@ -49,29 +50,20 @@ def _gpu_search(G, x_cpu, w_cpu, group, n_grid=20):
                 h=h)
 
 
-def _check_codes(c, ref, frac=1e-3):
-    diff = np.abs(c.astype(np.int64) - ref.astype(np.int64))
-    assert diff.max(initial=0) <= 1
-    assert np.mean(diff != 0) <= frac
-
-
 def _check_against_oracle(r, x, w, group):
     xf = x.float().numpy().astype(np.float64)
     wf = w.numpy().astype(np.float64)
     sx = A.channel_scale(xf)
     np.testing.assert_array_equal(r["sx"], sx)
-    ref = A.search(wf, O.hessian(xf), sx, 4, group, dtype=np.float32)
+    ref = A.search(wf, O.hessian(xf), sx, 4, group)
     np.testing.assert_allclose(r["losses"], ref["losses"], rtol=LOSS_RTOL)
     if r["best"] != ref["best"]:
         a, b = ref["losses"][r["best"]], ref["losses"][ref["best"]]
         assert abs(a - b) <= LOSS_RTOL * b, "a different alpha, not a near tie"
-    s = A.scales_for(sx, ref["alphas"][r["best"]], np.float32)
-    np.testing.assert_array_equal(r["s"], s)
-    q = A.quantize_scaled(wf, s, 4, group, np.float32)
-    _check_codes(r["codes"], q["codes"])
-    _check_codes(r["zeros"], q["zeros"])
-    same = (r["zeros"] == q["zeros"])
-    np.testing.assert_allclose(r["scales"][same], q["scales"][same], rtol=1e-6)
+    s = A.scales_for(sx, ref["alphas"][r["best"]])
+    np.testing.assert_array_equal(r["s"], s.astype(np.float32))
+    q = A.quantize_scaled(wf, s, 4, group)
+    check_layer(r["codes"], r["scales"], r["zeros"], q["codes"], q["scales"], q["zeros"], 0)
     return ref
 
 
@@ -114,9 +106,9 @@ def test_awq_full_size_q_proj(G):
     h = O.hessian(xf)
     alphas = A.alpha_grid()
     for a in sorted({0, r["best"]}):
-        q = A.quantize_scaled(wf, A.scales_for(sx, alphas[a], np.float32), 4, 128, np.float32)
+        q = A.quantize_scaled(wf, A.scales_for(sx, alphas[a]), 4, 128)
         ref = O.layer_loss_hessian(wf, q["w_hat"], h)
         assert r["losses"][a] == pytest.approx(ref, rel=LOSS_RTOL)
     assert r["losses"][r["best"]] == r["losses"].min()
-    np.testing.assert_array_equal(r["s"], A.scales_for(sx, alphas[r["best"]], np.float32))
-    _check_codes(r["codes"], q["codes"])
+    np.testing.assert_array_equal(r["s"], A.scales_for(sx, alphas[r["best"]]).astype(np.float32))
+    check_layer(r["codes"], r["scales"], r["zeros"], q["codes"], q["scales"], q["zeros"], 0)

@@ -50,7 +50,7 @@ def test_one_rank_sequence_equals_the_direct_calls(G):
     codes2 = O.unpack_codes(q2.cpu().numpy().view(np.uint32), 4, 512)
     assert np.mean(codes != codes2) <= 1e-3
     ref = O.gptq(w.cpu().numpy().astype(np.float64), O.hessian(x.cpu().float().numpy()), bits=4,
-                 group=128, sym=False, block=128, damp_rel=0.01, dtype=np.float32)
+                 group=128, sym=False, block=128, damp_rel=0.01)
     diff = np.abs(codes - ref["codes"])
     assert diff.max() <= 1 and np.mean(diff != 0) <= 1e-3
 

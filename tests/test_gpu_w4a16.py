@@ -94,7 +94,7 @@ def test_w4a16_oracle_quantized_layer(G):
     spec = synth.tiny_spec(96, 512, 2048, seed=5).with_(group=128)
     w = synth.gen_weight(spec).numpy().astype(np.float64)
     ref = O.gptq(w, O.hessian(synth.gen_tokens(spec).float().numpy()), bits=4,
-                 group=128, sym=False, block=128, damp_rel=0.01, dtype=np.float32)
+                 group=128, sym=False, block=128, damp_rel=0.01)
     words = torch.from_numpy(O.pack_codes(ref["codes"], 4).view(np.int32))
     scales = torch.from_numpy(np.asarray(ref["scales"], np.float32))
     zeros = torch.from_numpy(np.asarray(ref["zeros"]).astype(np.uint8))
