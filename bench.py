@@ -1,15 +1,30 @@
 #!/usr/bin/env python
 """GPTQ layer quantization throughput on B200: weights quantized per second.
 
-One step = the whole GPTQ path for one LLaMA-7B-shaped q_proj layer
-(W 4096x4096, 262144 calibration tokens, 4-bit asymmetric, one scale per
-output channel, B = 128): zero H, accumulate H = 2 X X^T over all tokens,
-damp + factor to G, quantize + pack all columns.  Inputs are resident in HBM
-when the timed region starts (X is 2.1 GB, larger than L2).  With N GPUs
-every rank quantizes its own independent layer (weak scaling, no collective
-on the data path).
+One step = the whole GPTQ path for one workload.  For every calibration
+input: zero H, accumulate H = 2 X X^T over all of its tokens, damp and
+factor H into G.  For every linear layer fed by that input: quantize and
+pack all of its columns with that G.  Inputs are resident in HBM when the
+timed region starts; every X is larger than L2.  With N GPUs every rank runs
+its own independent copy of the workload (weak scaling, no collective on
+the data path).
+
+Workloads (``--workload``; ``--bits`` overrides the code width):
+
+    down_proj_65b  (default) LLaMA-65B-shaped down projection: W 8192 x 22016,
+                   131072 tokens (H of 22016^2), 4-bit asymmetric, g = 128
+    mlp_65b        the 65B-shaped MLP: gate and up 22016 x 8192 sharing one
+                   input (H of 8192^2) plus the down projection; 2 Hessians,
+                   3 layers
+    block_7b       all 7 layers of a LLaMA-7B-shaped decoder block, g = 128:
+                   q/k/v share one input, gate/up another, o and down have
+                   their own; 4 Hessians, 7 layers
+    down_proj_7b   W 4096 x 11008, 262144 tokens, 4-bit g = 128
+    q_proj         W 4096 x 4096, 262144 tokens, 4-bit, one scale per row
+    small          W 256 x 256, 2048 tokens (a parity case)
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--bits B] [--sym]
 
 Prints one JSON line (rank 0).  Other measurements of the same library, each
 its own JSON line:
@@ -19,7 +34,6 @@ its own JSON line:
     --awq            the AWQ scale search on the q_proj layer, 32768 tokens
     --shard-layer    one q_proj layer strong-scaled across the ranks
                      (token-sharded H + all-reduce, row-sharded quantize)
-    --bits N, --sym  other code widths / the symmetric quantizer, same path
 """
 from __future__ import annotations
 
@@ -42,15 +56,17 @@ METRIC = "GPTQ weights quantized/s per linear layer"
 UNIT = "weights/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
                   "bf16_tflops_sustained": 1400.0}
+WORKLOADS = ("down_proj_65b", "mlp_65b", "block_7b", "down_proj_7b", "q_proj", "small")
+SM_COUNT = 148
 
 
-def parse_args():
+def parse_args(argv=None):
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=100)
-    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", choices=["q_proj", "small"], default="q_proj")
+    p.add_argument("--workload", choices=WORKLOADS, default="down_proj_65b")
     p.add_argument("--tokens", type=int, default=0,
                    help="calibration tokens (default: the workload's); a smaller "
                         "full-path configuration for profiling captures")
@@ -70,14 +86,78 @@ def parse_args():
                         "with 32768 calibration tokens, 4-bit g128")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    return p.parse_args()
+    return p.parse_args(argv)
+
+
+# ---------------------------------------------------------------- workloads
+def workload_layers(name: str, rank: int = 0, bits: int = 0, sym: bool = False,
+                    tokens: int = 0):
+    """The workload's layers grouped by calibration input: a list of groups,
+    each a list of layer specs that share one X (and so one H and one G).
+    Rank r of a weak-scaling run gets its own seeds for every W and X."""
+    from post_weight_quantization_26_b200 import synth
+    b = bits or 4
+    table = {
+        "small": lambda: [(synth.SMALL_256, 0)],
+        "q_proj": lambda: [(synth.Q_PROJ_7B, 0)],
+        "down_proj_7b": lambda: [(synth.DOWN_PROJ_7B, 0)],
+        "block_7b": lambda: synth.decoder_block_7b(b),
+        "mlp_65b": lambda: synth.mlp_65b(b),
+        "down_proj_65b": lambda: [synth.mlp_65b(b)[2]],
+    }
+    groups: dict[int, list] = {}
+    for spec, xin in table[name]():
+        spec = spec.with_(w_seed=spec.w_seed + rank, x_seed=spec.x_seed + 100 * rank)
+        if bits:
+            spec = spec.with_(bits=bits)
+        if sym:
+            spec = spec.with_(sym=True)
+        if tokens:
+            spec = spec.with_(n_tokens=tokens)
+        groups.setdefault(xin, []).append(spec)
+    return list(groups.values())
 
 
 def workload_spec(name: str, rank: int):
-    from post_weight_quantization_26_b200 import synth
-    base = synth.Q_PROJ_7B if name == "q_proj" else synth.SMALL_256
-    # weak scaling: every rank gets its own independent layer
-    return base.with_(w_seed=base.w_seed + rank, x_seed=base.x_seed + 100 * rank)
+    """The first layer of a workload (the only one for single-layer workloads)."""
+    return workload_layers(name, rank)[0][0]
+
+
+def work_model(groups):
+    """Algorithmic work of one step (per stage), counted as the method needs
+    it: the SYRK d(d+1)n flops per input, the factorization 2/3 d^3 fp64 flops
+    per input, the column sweep d_row d_col (d_col - 1) fp32 flops per layer,
+    and the packed output d_row d_col (1 + b/8) bytes per layer."""
+    w = {"weights": 0, "syrk_flops": 0.0, "chol_flops": 0.0, "prop_flops": 0.0,
+         "pack_bytes": 0.0}
+    for layers in groups:
+        d, n = layers[0].d_col, layers[0].n_tokens
+        w["syrk_flops"] += float(d) * (d + 1) * n
+        w["chol_flops"] += 2.0 / 3.0 * float(d) ** 3
+        for s in layers:
+            w["weights"] += s.d_row * s.d_col
+            w["prop_flops"] += float(s.d_row) * s.d_col * (s.d_col - 1)
+            w["pack_bytes"] += float(s.d_row) * s.d_col * (1 + s.bits / 8)
+    return w
+
+
+def workload_config(name, groups, world):
+    layers = [s for g in groups for s in g]
+    first = layers[0]
+    x_bytes = sum(g[0].n_tokens * g[0].d_col * 2 for g in groups)
+    cfg = {"workload": name if len(layers) > 1 else first.name,
+           "layers": [f"{s.name} {s.d_row}x{s.d_col}" for s in layers],
+           "inputs": len(groups),
+           "bits": first.bits, "group_size": first.group, "sym": first.sym,
+           "block": first.block, "damp": first.damp,
+           "w": f"{first.w_dist} sigma={first.w_sigma} {'bf16' if first.w_bf16 else 'fp32'}",
+           "x": "; ".join(f"{g[0].x_dist} bf16 {g[0].n_tokens} tokens x {g[0].d_col}, "
+                          f"{g[0].outlier_count} channels x{g[0].outlier_scale:g}" for g in groups),
+           "l2": "inputs larger than L2 (X bf16 %.2f GB per step)" % (x_bytes / 1e9),
+           "parallelism": f"{world} independent workload copy(ies), one per GPU"}
+    if len(layers) == 1:
+        cfg.update(d_row=first.d_row, d_col=first.d_col, n_tokens=first.n_tokens)
+    return cfg
 
 
 def load_peaks():
@@ -150,31 +230,50 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+
+
 # --------------------------------------------------------- oracle baseline
-def oracle_sample(spec, x_host, w_host, tokens=8192, rows=32):
-    """Time the CPU oracle on a bounded sample of the workload and scale to
-    one full layer: Hessian on a token prefix (scaled by n / prefix), the full
-    fp64 factorization, GPTQ on a subset of rows (scaled by d_row / rows)."""
+def oracle_sample(groups, x_hosts, w_hosts, tokens, fac_dim, rows):
+    """Time the CPU oracle, as it stands, on a bounded sample of the workload
+    and extrapolate to the whole step.  The sample is the leading
+    sub-problem: the first fac input channels, a token prefix and a few rows.
+    Per input: the Hessian of the prefix over those channels (time scaled by
+    n / prefix x (d / fac)^2) and its factorization (scaled by (d / fac)^3).
+    Per layer: GPTQ of `rows` rows over those fac columns with that factor
+    (scaled by d_row / rows x d_col / fac: linear in the width, which
+    under-counts the oracle's O(d_col^2) trailing updates, so the estimate
+    favours the oracle).  Returns the extrapolated seconds per step, the
+    seconds the sample itself took, per-stage estimates, and a description."""
     import numpy as np
 
     from oracle import gptq_oracle as O
-    t0 = time.perf_counter()
-    xs = x_host[:tokens].float().numpy()
-    h = O.hessian(xs)
-    t_h = time.perf_counter() - t0
-    t0 = time.perf_counter()
-    hd, dead = O.dampen(h, spec.damp)
-    u = O.hinv_cholesky_upper(hd)
-    t_f = time.perf_counter() - t0
-    t0 = time.perf_counter()
-    O.gptq_quantize(w_host[:rows].numpy().astype(np.float64), u, spec.bits, spec.group,
-                    spec.sym, spec.block, dead=dead)
-    t_q = time.perf_counter() - t0
-    total = t_h * spec.n_tokens / tokens + t_f + t_q * spec.d_row / rows
-    return {"seconds_per_layer": total, "hessian_s": t_h, "factor_s": t_f, "quant_s": t_q,
-            "sample": (f"H on {tokens} of {spec.n_tokens} tokens (x{spec.n_tokens / tokens:g}), "
-                       f"full {spec.d_col}^2 fp64 factorization, GPTQ on {rows} of "
-                       f"{spec.d_row} rows (x{spec.d_row / rows:g})")}
+    est = {"hessian": 0.0, "factor": 0.0, "quantize": 0.0}
+    t_all = time.perf_counter()
+    parts = []
+    for gi, layers in enumerate(groups):
+        d, n = layers[0].d_col, layers[0].n_tokens
+        tk, fac = min(tokens, n), min(fac_dim, d)
+        t0 = time.perf_counter()
+        h = O.hessian(x_hosts[gi][:tk, :fac].float().numpy())
+        est["hessian"] += (time.perf_counter() - t0) * (n / tk) * (d / fac) ** 2
+        t0 = time.perf_counter()
+        hd, dead = O.dampen(h, layers[0].damp)
+        u = O.hinv_cholesky_upper(hd)
+        est["factor"] += (time.perf_counter() - t0) * (d / fac) ** 3
+        for li, s in enumerate(layers):
+            r = min(rows, s.d_row)
+            w = w_hosts[gi][li][:r, :fac].numpy().astype(np.float64)
+            t0 = time.perf_counter()
+            O.gptq_quantize(w, u, s.bits, s.group, s.sym, s.block, dead=dead)
+            est["quantize"] += (time.perf_counter() - t0) * (s.d_row / r) * (d / fac)
+        parts.append(f"H over the first {fac} of {d} channels on {tk} of {n} tokens, its "
+                     f"factor, GPTQ of {min(rows, layers[0].d_row)} rows x {fac} columns "
+                     f"per layer ({len(layers)} layer(s))")
+    sample_s = time.perf_counter() - t_all
+    return {"seconds_per_step": sum(est.values()), "sample_seconds": sample_s,
+            "stage_s": est,
+            "sample": "; ".join(parts) + "; extrapolated: H x n/prefix x (d/fac)^2, factor x "
+                      "(d/fac)^3, GPTQ x rows x width (linear)"}
 
 
 def cpu_cores():
@@ -187,36 +286,57 @@ def cpu_cores():
         return cores
 
 
+def host_inputs(groups, pin=False):
+    """Seeded host inputs: one token-major bf16 X per input group, one fp32 W
+    per layer (pinned when asked, for the device copies)."""
+    import torch
+
+    from post_weight_quantization_26_b200 import synth
+    xs, ws = [], []
+    for layers in groups:
+        s0 = layers[0]
+        x = torch.empty((s0.n_tokens, s0.d_col), dtype=torch.bfloat16)
+        if pin:
+            x = x.pin_memory()
+        synth.gen_tokens(s0, out=x)
+        xs.append(x)
+        ws.append([synth.gen_weight(s).pin_memory() if pin else synth.gen_weight(s)
+                   for s in layers])
+    return xs, ws
+
+
 # --------------------------------------------------------------- reference
 def run_reference(args, rank, world):
+    """The oracle arm: the CPU oracle timed on the host cores on a bounded
+    sample of every step (rank 0 only).  `ms_per_step` is the time the sample
+    took; `value` is the whole-step rate extrapolated from it."""
     if rank != 0:
         return
+    groups = workload_layers(args.workload, 0, args.bits, args.sym, args.tokens)
+    tokens, fac, rows = 1024, 4096, 8
     from post_weight_quantization_26_b200 import synth
-    spec = workload_spec(args.workload, 0)
-    if args.bits:
-        spec = spec.with_(bits=args.bits, name=f"{spec.name}_int{args.bits}")
-    if args.sym:
-        spec = spec.with_(sym=True, name=f"{spec.name}_sym")
-    tokens = min(8192, spec.n_tokens)
-    x_host = synth.gen_tokens(spec, 0, tokens)
-    w_host = synth.gen_weight(spec)
-    times = []
+    xs = [synth.gen_tokens(g[0], 0, min(tokens, g[0].n_tokens)) for g in groups]
+    ws = [[synth.gen_weight(s.with_(d_row=min(rows, s.d_row))) for s in g] for g in groups]
+    est, sample_s = [], []
     res = None
     for i in range(args.warmup + args.steps):
-        res = oracle_sample(spec, x_host, w_host, tokens=tokens)
+        res = oracle_sample(groups, xs, ws, tokens, fac, rows)
         if i >= args.warmup:
-            times.append(res["seconds_per_layer"])
-    sec = statistics.mean(times)
-    value = spec.d_row * spec.d_col / sec
+            est.append(res["seconds_per_step"])
+            sample_s.append(res["sample_seconds"])
+    sec = statistics.mean(est)
+    value = work_model(groups)["weights"] / sec
     cores = cpu_cores()
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(spec, world=1),
+        "ms_per_step": statistics.mean(sample_s) * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(args.workload, groups, 1),
+        "extrapolated": True,
+        "extrapolated_ms_per_step": sec * 1e3,
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": res["sample"]},
+                         "sample": res["sample"], "extrapolated": True},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -235,20 +355,11 @@ def max_over_ranks(ms: float, world: int, device) -> float:
     return float(t.item())
 
 
-def weak_value(world: int, d_row: int, d_col: int, ms_max: float) -> float:
-    """Whole-job weights/s: every rank quantizes its own d_row x d_col layer,
-    and the job takes as long as its slowest rank."""
-    return world * d_row * d_col / (ms_max / 1e3)
-
-
-def workload_config(spec, world):
-    return {"workload": spec.name, "d_row": spec.d_row, "d_col": spec.d_col,
-            "n_tokens": spec.n_tokens, "bits": spec.bits, "group_size": spec.group,
-            "sym": spec.sym, "block": spec.block, "damp": spec.damp,
-            "w": f"{spec.w_dist} sigma={spec.w_sigma} {'bf16' if spec.w_bf16 else 'fp32'}",
-            "x": f"{spec.x_dist} bf16, {spec.outlier_count} channels x{spec.outlier_scale:g}",
-            "l2": "inputs larger than L2 (X bf16 %.2f GB)" % (spec.n_tokens * spec.d_col * 2 / 1e9),
-            "parallelism": f"{world} independent layer(s), one per GPU"}
+def weak_value(world: int, weights: int, ms_max: float) -> float:
+    """Whole-job weights/s: every rank quantizes its own copy of the
+    workload's `weights` weights, and the job takes as long as its slowest
+    rank."""
+    return world * weights / (ms_max / 1e3)
 
 
 # ------------------------------------------------------------------- ours
@@ -268,13 +379,73 @@ def kernel_traffic(name: str, src_rel: str):
         return None
 
 
+def stage_roofline(work, stage_ms, ms, peaks, peak_src, clk, groups, name):
+    """Each stage against its own bound, the combined roofline T*, and the
+    roofline object of the stage that takes the most time."""
+    sm_mhz = (clk or {}).get("sm_mhz") or peaks.get("sm_max_mhz", 1965.0)
+    bf16 = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    fp64 = SM_COUNT * 64 * 2 * sm_mhz * 1e6 / 1e12
+    fp32 = SM_COUNT * 128 * 2 * sm_mhz * 1e6 / 1e12
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    t_star = (work["syrk_flops"] / (bf16 * 1e12) + work["chol_flops"] / (fp64 * 1e12)
+              + work["prop_flops"] / (fp32 * 1e12) + work["pack_bytes"] / (hbm * 1e9))
+    ach = {
+        "hessian": work["syrk_flops"] / (stage_ms["hessian"] / 1e3) / 1e12,
+        "prepare": work["chol_flops"] / (stage_ms["prepare"] / 1e3) / 1e12,
+        "quantize": work["prop_flops"] / (stage_ms["quantize"] / 1e3) / 1e12,
+    }
+    stages = {
+        "hessian": {"ms": stage_ms["hessian"], "tflops": ach["hessian"],
+                    "frac": ach["hessian"] / bf16,
+                    "bound": f"tensor bf16 {bf16:.0f} TF/s (bf16_tflops of {peak_src})"},
+        "prepare": {"ms": stage_ms["prepare"], "tflops": ach["prepare"],
+                    "frac": ach["prepare"] / fp64,
+                    "bound": f"fp64 {fp64:.1f} TF/s derived: {SM_COUNT} SMs x 64 FMA/clk x 2 "
+                             f"at {sm_mhz:.0f} MHz"},
+        "quantize": {"ms": stage_ms["quantize"], "tflops": ach["quantize"],
+                     "frac": ach["quantize"] / fp32,
+                     "bound": f"fp32 {fp32:.1f} TF/s derived: {SM_COUNT} SMs x 128 FMA/clk x 2 "
+                              f"at {sm_mhz:.0f} MHz"},
+        "zero_h": {"ms": stage_ms["zero_h"]},
+        "combined_t_star_ms": t_star * 1e3,
+        "combined_frac": t_star * 1e3 / ms,
+    }
+    top = max(("hessian", "prepare", "quantize"), key=lambda k: stage_ms[k])
+    if top == "hessian":
+        single = len(groups) == 1
+        roof = {"bound": "tensor", "kernel": "syrk_bf16_tcgen05_kernel (the accumulate call's "
+                                             "only kernel)",
+                "achieved": ach["hessian"], "peak": bf16, "unit": "TFLOP/s",
+                "frac": ach["hessian"] / bf16,
+                "traffic": kernel_traffic(f"syrk_bf16_tcgen05_kernel/{name}",
+                                          "post_weight_quantization_26_b200/csrc/syrk_tcgen05.cuh")
+                if single else None,
+                "peak_source": f"bf16_tflops (burst) of {peak_src}"}
+    elif top == "prepare":
+        roof = {"bound": "tensor", "kernel": "dgemm_nt_kernel (fp64 MMA), over the whole "
+                                             "prepare stage (with leaf_kernel and the damping)",
+                "achieved": ach["prepare"], "peak": fp64, "unit": "TFLOP/s",
+                "frac": ach["prepare"] / fp64,
+                "traffic": kernel_traffic(f"dgemm_nt_kernel/{name}",
+                                          "post_weight_quantization_26_b200/csrc/chol_fp64.cuh"),
+                "peak_source": f"derived: {SM_COUNT} SMs x 64 fp64 FMA/clk x 2 at the sampled "
+                               f"{sm_mhz:.0f} MHz (no measured fp64 peak)"}
+    else:
+        roof = {"bound": "alu", "kernel": "block_step_kernel + trailing_tf32x3_kernel, over the "
+                                          "whole quantize stage",
+                "achieved": ach["quantize"], "peak": fp32, "unit": "TFLOP/s",
+                "frac": ach["quantize"] / fp32, "traffic": None,
+                "peak_source": f"derived: {SM_COUNT} SMs x 128 fp32 FMA/clk x 2 at the sampled "
+                               f"{sm_mhz:.0f} MHz"}
+    return stages, roof
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
 
     from post_weight_quantization_26_b200 import build as _build
     from post_weight_quantization_26_b200 import gptq as G
-    from post_weight_quantization_26_b200 import synth
 
     if rank == 0:
         _build.build()
@@ -282,44 +453,46 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     G.load_library()
     dev = torch.device("cuda", local_rank)
-    spec = workload_spec(args.workload, rank)
-    if args.tokens:
-        spec = spec.with_(n_tokens=args.tokens, name=f"{spec.name}_n{args.tokens}")
-    if args.bits:
-        spec = spec.with_(bits=args.bits, name=f"{spec.name}_int{args.bits}")
-    if args.sym:
-        spec = spec.with_(sym=True, name=f"{spec.name}_sym")
-    d, n, dr = spec.d_col, spec.n_tokens, spec.d_row
-    cfg = G.make_config(bits=spec.bits, group_size=spec.group, sym=spec.sym,
-                        block=spec.block, damp_rel=spec.damp)
+    groups = workload_layers(args.workload, rank, args.bits, args.sym, args.tokens)
+    work = work_model(groups)
+    x_hosts, w_hosts = host_inputs(groups, pin=True)
 
-    x_host = torch.empty((n, d), dtype=torch.bfloat16).pin_memory()
-    synth.gen_tokens(spec, out=x_host)
-    w_host = synth.gen_weight(spec).pin_memory()
-    x = x_host.to(dev)
-    w = w_host.to(dev)
-    H = torch.zeros((d, d), dtype=torch.float32, device=dev)
-    Gm = torch.empty_like(H)
-    dead = torch.empty(d, dtype=torch.uint8, device=dev)
-    ws = G.alloc_workspace(dr, d, cfg, device=dev)
-    qw, sc, ze = G.alloc_outputs(dr, d, cfg, device=dev)
+    cfgs = [[G.make_config(bits=s.bits, group_size=s.group, sym=s.sym, block=s.block,
+                           damp_rel=s.damp) for s in layers] for layers in groups]
+    ws_bytes = max(G.gptq_workspace_size(s.d_row, s.d_col, c)
+                   for layers, cl in zip(groups, cfgs) for s, c in zip(layers, cl))
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    dev_in = []
+    for gi, layers in enumerate(groups):
+        d = layers[0].d_col
+        H = torch.zeros((d, d), dtype=torch.float32, device=dev)
+        dev_in.append({
+            "x": x_hosts[gi].to(dev), "H": H, "G": torch.empty_like(H),
+            "dead": torch.empty(d, dtype=torch.uint8, device=dev),
+            "w": [wh.to(dev) for wh in w_hosts[gi]],
+            "out": [G.alloc_outputs(s.d_row, s.d_col, c, device=dev)
+                    for s, c in zip(layers, cfgs[gi])]})
     stream = torch.cuda.current_stream(dev)
 
-    def step(ev=None):
-        if ev:
-            ev[0].record(stream)
-        H.zero_()
-        if ev:
-            ev[1].record(stream)
-        G.gptq_hessian_accumulate(H, x)
-        if ev:
-            ev[2].record(stream)
-        G.gptq_prepare_hinv(H, spec.damp, Gm, dead, ws)
-        if ev:
-            ev[3].record(stream)
-        G.gptq_quantize_layer(w, Gm, dead, cfg, qw, sc, ze, ws)
-        if ev:
-            ev[4].record(stream)
+    def step(marks=None):
+        def mark(stage):
+            if marks is not None:
+                e = torch.cuda.Event(enable_timing=True)
+                e.record(stream)
+                marks.append((stage, e))
+        mark("start")
+        for gi, layers in enumerate(groups):
+            b = dev_in[gi]
+            b["H"].zero_()
+            mark("zero_h")
+            G.gptq_hessian_accumulate(b["H"], b["x"])
+            mark("hessian")
+            G.gptq_prepare_hinv(b["H"], layers[0].damp, b["G"], b["dead"], ws)
+            mark("prepare")
+            for li, s in enumerate(layers):
+                qw, sc, ze = b["out"][li]
+                G.gptq_quantize_layer(b["w"][li], b["G"], b["dead"], cfgs[gi][li], qw, sc, ze, ws)
+                mark("quantize")
 
     for _ in range(args.warmup):
         step()
@@ -327,7 +500,7 @@ def run_ours(args, rank, world, local_rank):
     if G.gptq_device_status() != 0:
         raise RuntimeError("device status set during warm-up")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    marks = [[] for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local_rank)
     if world > 1:
@@ -337,7 +510,7 @@ def run_ours(args, rank, world, local_rank):
     launches0 = G.gptq_launch_count()
     t0.record(stream)
     for i in range(args.steps):
-        step(evs[i])
+        step(marks[i])
     t1.record(stream)
     torch.cuda.synchronize(dev)
     launches = G.gptq_launch_count() - launches0
@@ -345,121 +518,91 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     ms = t0.elapsed_time(t1) / args.steps
-    stages = {"zero_h": [], "hessian": [], "prepare": [], "quantize": []}
-    for e in evs:
-        stages["zero_h"].append(e[0].elapsed_time(e[1]))
-        stages["hessian"].append(e[1].elapsed_time(e[2]))
-        stages["prepare"].append(e[2].elapsed_time(e[3]))
-        stages["quantize"].append(e[3].elapsed_time(e[4]))
-    stage_ms = {k: statistics.mean(v) for k, v in stages.items()}
+    stage_ms = {k: 0.0 for k in ("zero_h", "hessian", "prepare", "quantize")}
+    for m in marks:
+        for (_, a), (stage, b) in zip(m[:-1], m[1:]):
+            stage_ms[stage] += a.elapsed_time(b) / args.steps
     if G.gptq_device_status() != 0:
         raise RuntimeError("device status set during the timed region")
 
     ms_max = max_over_ranks(ms, world, dev)
-    value = weak_value(world, dr, d, ms_max)
+    value = weak_value(world, work["weights"], ms_max)
 
     # ---- end to end: host buffers in, host buffers out, through the same API
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, G, spec, cfg, x_host, w_host, dev, stream, world)
+        e2e = run_e2e(args, G, groups, cfgs, x_hosts, w_hosts, dev_in, ws, dev, stream, world,
+                      work["weights"])
 
     if rank != 0:
         return
     peaks, peak_src = load_peaks()
-    syrk_s = stage_ms["hessian"] / 1e3
-    syrk_flops = d * (d + 1) * n
-    achieved = syrk_flops / syrk_s / 1e12
-    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
-    traffic = kernel_traffic("syrk_bf16_tcgen05_kernel",
-                             "post_weight_quantization_26_b200/csrc/syrk_tcgen05.cuh")
-    roofline = {"bound": "tensor", "kernel": "syrk_bf16_tcgen05_kernel",
-                "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": traffic,
-                "peak_source": f"bf16_tflops_sustained of {peak_src}"}
-    # other stages against their own bounds (SM clock from the sampled median)
-    sm_mhz = (clk or {}).get("sm_mhz") or peaks.get("sm_max_mhz", 1965.0)
-    fp64_peak = 148 * 64 * 2 * sm_mhz * 1e6 / 1e12
-    fp32_peak = 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
-    chol_flops = 2.0 / 3.0 * d ** 3
-    prop_flops = dr * d * (d - 1)
-    t_star = (syrk_flops / (peak * 1e12) + chol_flops / (fp64_peak * 1e12)
-              + prop_flops / (fp32_peak * 1e12)
-              + dr * d * (1 + spec.bits / 8) / (peaks.get("hbm_gbs", 6650.0) * 1e9))
-    stage_roofline = {
-        "hessian": {"ms": stage_ms["hessian"], "frac": achieved / peak, "bound": "tensor bf16"},
-        "prepare": {"ms": stage_ms["prepare"],
-                    "frac": chol_flops / (stage_ms["prepare"] / 1e3) / 1e12 / fp64_peak,
-                    "bound": f"alu fp64 {fp64_peak:.1f} TF/s at {sm_mhz:.0f} MHz"},
-        "quantize": {"ms": stage_ms["quantize"],
-                     "frac": prop_flops / (stage_ms["quantize"] / 1e3) / 1e12 / fp32_peak,
-                     "bound": f"alu fp32 {fp32_peak:.1f} TF/s at {sm_mhz:.0f} MHz"},
-        "zero_h": {"ms": stage_ms["zero_h"]},
-        "combined_t_star_ms": t_star * 1e3,
-        "combined_frac": t_star * 1e3 / ms,
-    }
+    stages, roofline = stage_roofline(work, stage_ms, ms, peaks, peak_src, clk, groups,
+                                      args.workload)
     cpu = None
     if not args.no_cpu_baseline and world == 1:
-        res = oracle_sample(spec, x_host, w_host, tokens=min(8192, n))
-        cpu = {"value": dr * d / res["seconds_per_layer"], "unit": UNIT, "cores": cpu_cores(),
-               "kind": "oracle", "sample": res["sample"],
-               "stage_s": {"hessian_full_est": res["hessian_s"] * n / min(8192, n),
-                           "factor": res["factor_s"], "quant_full_est": res["quant_s"] * dr / 32}}
+        res = oracle_sample(groups, x_hosts, w_hosts, tokens=4096, fac_dim=8192, rows=32)
+        cpu = {"value": work["weights"] / res["seconds_per_step"], "unit": UNIT,
+               "cores": cpu_cores(), "kind": "oracle", "sample": res["sample"],
+               "extrapolated": True, "sample_seconds": res["sample_seconds"],
+               "stage_s_est": res["stage_s"]}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16 in / f32 acc (H); f64 (factor); f32 (sweep)",
-        "data": "synthetic (seeded LLaMA-7B-shaped layer and activations)",
-        "config": workload_config(spec, world),
-        "stage_ms": stage_ms, "stages": stage_roofline,
+        "data": "synthetic (seeded LLaMA-shaped layers and activations)",
+        "config": workload_config(args.workload, groups, world),
+        "stage_ms": stage_ms, "stages": stages,
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": launches, "clocks": clk,
     }
     print(json.dumps(line), flush=True)
 
 
-def run_e2e(args, G, spec, cfg, x_host, w_host, dev, stream, world):
+def run_e2e(args, G, groups, cfgs, x_hosts, w_hosts, dev_in, ws, dev, stream, world, weights):
     """Same metric through the public API with host buffers: every step copies
-    X (in chunks, overlapped with the accumulation on a copy stream) and W
-    from pinned host memory and reads the packed result back to the host."""
+    each X (in chunks, overlapped with the accumulation on a copy stream) and
+    each W from pinned host memory, and reads the packed results back to the
+    host."""
     import torch
     import torch.distributed as dist
-    d, n, dr = spec.d_col, spec.n_tokens, spec.d_row
     chunk = 32768
-    stage = [torch.empty((chunk, d), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    dmax = max(layers[0].d_col for layers in groups)
+    stage = [torch.empty((chunk * dmax,), dtype=torch.bfloat16, device=dev) for _ in range(2)]
     copy_stream = torch.cuda.Stream(dev)
-    H = torch.zeros((d, d), dtype=torch.float32, device=dev)
-    Gm = torch.empty_like(H)
-    dead = torch.empty(d, dtype=torch.uint8, device=dev)
-    ws = G.alloc_workspace(dr, d, cfg, device=dev)
-    qw, sc, ze = G.alloc_outputs(dr, d, cfg, device=dev)
-    w = torch.empty((dr, d), dtype=torch.float32, device=dev)
-    qh = torch.empty(qw.shape, dtype=qw.dtype).pin_memory()
-    sh = torch.empty(sc.shape, dtype=sc.dtype).pin_memory()
-    zh = torch.empty(ze.shape, dtype=ze.dtype).pin_memory()
+    host_out = [[tuple(torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in o)
+                 for o in b["out"]] for b in dev_in]
     copied = [torch.cuda.Event() for _ in range(2)]
     consumed = [torch.cuda.Event() for _ in range(2)]
 
     def step():
-        H.zero_()
-        w.copy_(w_host, non_blocking=True)
-        nchunks = (n + chunk - 1) // chunk
-        for i in range(nchunks):
-            b = i & 1
-            a, e = i * chunk, min(n, (i + 1) * chunk)
-            with torch.cuda.stream(copy_stream):
-                if i >= 2:
-                    copy_stream.wait_event(consumed[b])
-                stage[b][: e - a].copy_(x_host[a:e], non_blocking=True)
-                copied[b].record(copy_stream)
-            stream.wait_event(copied[b])
-            G.gptq_hessian_accumulate(H, stage[b][: e - a])
-            consumed[b].record(stream)
-        G.gptq_prepare_hinv(H, spec.damp, Gm, dead, ws)
-        G.gptq_quantize_layer(w, Gm, dead, cfg, qw, sc, ze, ws)
-        qh.copy_(qw, non_blocking=True)
-        sh.copy_(sc, non_blocking=True)
-        zh.copy_(ze, non_blocking=True)
+        it = 0
+        for gi, layers in enumerate(groups):
+            b = dev_in[gi]
+            d, n = layers[0].d_col, layers[0].n_tokens
+            b["H"].zero_()
+            for li in range(len(layers)):
+                b["w"][li].copy_(w_hosts[gi][li], non_blocking=True)
+            for a in range(0, n, chunk):
+                e = min(n, a + chunk)
+                k = it & 1
+                buf = stage[k][: (e - a) * d].view(e - a, d)
+                with torch.cuda.stream(copy_stream):
+                    if it >= 2:
+                        copy_stream.wait_event(consumed[k])
+                    buf.copy_(x_hosts[gi][a:e], non_blocking=True)
+                    copied[k].record(copy_stream)
+                stream.wait_event(copied[k])
+                G.gptq_hessian_accumulate(b["H"], buf)
+                consumed[k].record(stream)
+                it += 1
+            G.gptq_prepare_hinv(b["H"], layers[0].damp, b["G"], b["dead"], ws)
+            for li, s in enumerate(layers):
+                qw, sc, ze = b["out"][li]
+                G.gptq_quantize_layer(b["w"][li], b["G"], b["dead"], cfgs[gi][li], qw, sc, ze, ws)
+                for h, t in zip(host_out[gi][li], b["out"][li]):
+                    h.copy_(t, non_blocking=True)
 
     steps = max(1, args.steps)
     for _ in range(max(1, min(args.warmup, 3))):
@@ -474,9 +617,10 @@ def run_e2e(args, G, spec, cfg, x_host, w_host, dev, stream, world):
     t1.record(stream)
     torch.cuda.synchronize(dev)
     ms = max_over_ranks(t0.elapsed_time(t1) / steps, world, dev)
-    h2d = n * d * 2 + dr * d * 4
-    d2h = qw.numel() * 4 + sc.numel() * 4 + ze.numel()
-    return {"value": weak_value(world, dr, d, ms), "unit": UNIT, "ms_per_step": ms,
+    h2d = sum(g[0].n_tokens * g[0].d_col * 2 + sum(s.d_row * s.d_col * 4 for s in g)
+              for g in groups)
+    d2h = sum(t.numel() * t.element_size() for b in dev_in for o in b["out"] for t in o)
+    return {"value": weak_value(world, weights, ms), "unit": UNIT, "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
 # ------------------------------------------------- dequant-fused matmul

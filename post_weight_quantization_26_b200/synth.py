@@ -180,6 +180,18 @@ def _chunk(spec: LayerSpec, i: int, idx: torch.Tensor) -> torch.Tensor:
     return x.to(torch.bfloat16)
 
 
+def _free_host_bytes() -> float:
+    """Available host memory in bytes (48 GB if it cannot be read)."""
+    try:
+        with open("/proc/meminfo") as f:
+            for line in f:
+                if line.startswith("MemAvailable:"):
+                    return float(line.split()[1]) * 1024.0
+    except OSError:
+        pass
+    return 48e9
+
+
 def gen_tokens(spec: LayerSpec, t0: int = 0, t1: int | None = None,
                out: torch.Tensor | None = None,
                threads: int | None = None) -> torch.Tensor:
@@ -205,9 +217,10 @@ def gen_tokens(spec: LayerSpec, t0: int = 0, t1: int | None = None,
         out[lo - t0: hi - t0].copy_(x[lo - i * CHUNK: hi - i * CHUNK])
 
     chunks = list(range(c0, c1 + 1))
-    # one chunk's fp32 draws take ~3 x CHUNK x d_col x 4 bytes while in flight
+    # one chunk's fp32 draws take ~3 x CHUNK x d_col x 4 bytes while in flight;
+    # the chunks in flight may use up to a quarter of the free host memory
     cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
-    by_mem = max(1, int(12e9 // (3 * CHUNK * spec.d_col * 4)))
+    by_mem = max(1, int(_free_host_bytes() // 4 // (3 * CHUNK * spec.d_col * 4)))
     nthreads = threads or min(len(chunks), max(1, cores), by_mem)
     if nthreads <= 1 or len(chunks) == 1:
         for i in chunks:

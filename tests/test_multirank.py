@@ -35,7 +35,7 @@ def _worker(rank, world, port, q):
         ms = 10.0 + 5.0 * rank           # rank 1 is the slow one
         ms_max = bench.max_over_ranks(ms, world, torch.device("cpu"))
         spec = bench.workload_spec("q_proj", rank)
-        value = bench.weak_value(world, spec.d_row, spec.d_col, ms_max)
+        value = bench.weak_value(world, spec.d_row * spec.d_col, ms_max)
         q.put((rank, ms_max, spec.w_seed, spec.x_seed, value))
     finally:
         dist.destroy_process_group()
@@ -62,7 +62,7 @@ def test_single_rank_needs_no_process_group():
     sys.path.insert(0, ROOT)
     import bench
     assert bench.max_over_ranks(3.5, 1, None) == 3.5
-    assert bench.weak_value(1, 10, 20, 2.0) == pytest.approx(100000.0)
+    assert bench.weak_value(1, 200, 2.0) == pytest.approx(100000.0)
 
 
 def _reference_arm(rank, world):
@@ -84,3 +84,21 @@ def test_reference_arm_runs_on_rank_zero_only():
     assert rec["impl"] == "reference" and rec["value"] > 0
     assert rec["cpu_baseline"]["kind"] == "oracle"
     assert rec["e2e"]["h2d_bytes_per_step"] == 0
+    assert rec["extrapolated"] is True and rec["cpu_baseline"]["extrapolated"] is True
+
+
+def test_workloads_group_layers_by_input():
+    sys.path.insert(0, ROOT)
+    import bench
+    block = bench.workload_layers("block_7b", bits=3)
+    assert [len(g) for g in block] == [3, 1, 2, 1]          # qkv, o, gate/up, down
+    assert all(s.bits == 3 and s.group == 128 for g in block for s in g)
+    assert len({s.x_seed for s in block[0]}) == 1
+    w = bench.work_model(block)
+    assert w["weights"] == 4 * 4096 * 4096 + 2 * 11008 * 4096 + 4096 * 11008
+    mlp = bench.workload_layers("mlp_65b", rank=1)
+    assert [len(g) for g in mlp] == [2, 1]
+    assert mlp[0][0].w_seed == 1 and mlp[0][0].x_seed == 101   # rank 1's own seeds
+    down = bench.workload_layers("down_proj_65b")
+    assert [(s.d_row, s.d_col, s.n_tokens, s.group) for g in down for s in g] == \
+        [(8192, 22016, 131072, 128)]
