@@ -19,6 +19,12 @@
 //   U_k      A_ij -= L_ik L_jk^T on the other lower tiles (i, j > k) and
 //            Mt[:k+1, i] -= Mt[:k+1, k] L_ik^T for the rows i > k, on all
 //            SMs but two, so that D_k and the serial leaf run beside it.
+// The trailing updates are lazy over windows of m panels (window_panels):
+// inside a window U_k and D_k apply panel k only to the window's remaining
+// columns; the window's last panel applies all m panels (K = 128 m) to
+// everything right of the window.  Same sums, regrouped, so most of the
+// 2/3 d^3 flops run with a 4x longer K per output tile and a quarter of the
+// trailing matrix's read-modify-write traffic.
 // Every product is an "NT" GEMM (both operands row-major along K) on the
 // fp64 MMA path (mma.sync m8n8k4 f64), staged by cp.async through a 3-deep
 // ring of padded shared-memory tiles.
@@ -30,6 +36,13 @@ namespace gptq {
 namespace chol {
 
 constexpr int NB = 128;  // panel / leaf width
+
+// Panels per lazy-update window (see gptq_prepare_hinv): the window's last
+// panel applies all of them to the trailing matrix at once (K = 128 m).
+#ifndef GPTQ_WINDOW_PANELS
+#define GPTQ_WINDOW_PANELS 4
+#endif
+inline int window_panels(int d) { return d >= 8192 ? GPTQ_WINDOW_PANELS : 1; }
 
 // -------------------------------------------------------------- damping
 // One CTA: mean of diag(H), dead channels, NaN/Inf check.

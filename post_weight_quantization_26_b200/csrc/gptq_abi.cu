@@ -610,6 +610,8 @@ gptq_status gptq_prepare_hinv(const float* H, int64_t d, double damp_rel, float*
   auto at = [&](double* m, int r, int c) { return m + static_cast<size_t>(r) * di + c; };
 
   GPTQ_CUDA_TRY(cudaMemsetAsync(pivot, 0xFF, 8, s));
+  // M^T accumulates its off-diagonal blocks from zero
+  GPTQ_CUDA_TRY(cudaMemsetAsync(Mt, 0, static_cast<size_t>(d) * d * 8, s));
   chol::diag_stats_kernel<<<1, 1024, 0, s>>>(H, di, damp_rel, dead_mask, stats, istat);
   GPTQ_LAUNCH_CHECK();
   {
@@ -629,10 +631,15 @@ gptq_status gptq_prepare_hinv(const float* H, int64_t d, double damp_rel, float*
   };
   leaf(0, std::min(NB, di), s);
   GPTQ_LAUNCH_CHECK();
-  // Step k: P_k (caller's stream) forms the panel and rescales M's row
+  // Step k: P_k (caller's stream) forms the panel and rescales M's column
   // block k; then the auxiliary stream updates the next diagonal block (D_k)
   // and factors it (leaf k+1) while the caller's stream runs the rest of the
-  // trailing update U_k; P_{k+1} waits for both.
+  // update U_k; P_{k+1} waits for both.  The trailing updates are lazy over
+  // windows of m panels: inside a window, U_k only updates the window's
+  // remaining columns (K = one panel); the window's last panel updates every
+  // column to its right with all m panels at once (K = 128 m), so most of the
+  // d^3 work runs with long K.  m = 1 is the plain right-looking sweep.
+  const int m = chol::window_panels(di);
   for (int k = 0; k < nt; ++k) {
     const int k0 = k * NB, nk = std::min(NB, di - k0), k1 = k0 + nk, rest = di - k1;
     double* Xk = Xd + static_cast<size_t>(k) * NB * NB;
@@ -656,15 +663,20 @@ gptq_status gptq_prepare_hinv(const float* H, int64_t d, double damp_rel, float*
     if (st != GPTQ_OK) return st;
     if (rest <= 0) break;
     const int n1 = std::min(NB, rest);  // next diagonal block
+    // window of this panel: columns [e0, e1); the panels applied now are
+    // [ka, k1) with K = kK, to the columns [k1, w1)
+    const int e0 = (k / m) * m * NB, e1 = std::min(di, e0 + m * NB);
+    const bool last = k1 >= e1;
+    const int ka = last ? e0 : k0, kK = k1 - ka, w1 = last ? di : e1;
     GPTQ_CUDA_TRY(cudaEventRecord(evP[k & 1], s));
     GPTQ_CUDA_TRY(cudaStreamWaitEvent(aux, evP[k & 1], 0));
     {
       std::vector<chol::GemmProblem> dk(1);
-      chol::GemmProblem& q = dk[0];  // D_k: A_{k+1,k+1} -= L_{k+1} L_{k+1}^T
+      chol::GemmProblem& q = dk[0];  // D_k: A_{k+1,k+1} -= L_{k+1,[ka,k1)} L_{k+1,[ka,k1)}^T
       q = chol::GemmProblem{};
-      q.A = at(A, k1, k0); q.lda = di; q.B = at(A, k1, k0); q.ldb = di;
+      q.A = at(A, k1, ka); q.lda = di; q.B = at(A, k1, ka); q.ldb = di;
       q.C = at(A, k1, k1); q.ldc = di;
-      q.M = n1; q.N = n1; q.K = nk; q.alpha = -1.0; q.beta = 1.0;
+      q.M = n1; q.N = n1; q.K = kK; q.alpha = -1.0; q.beta = 1.0;
       st = launch_nt<32, 1>(dk, aux);
       if (st != GPTQ_OK) return st;
       leaf(k1, n1, aux);
@@ -674,28 +686,31 @@ gptq_status gptq_prepare_hinv(const float* H, int64_t d, double damp_rel, float*
     std::vector<chol::GemmProblem> uk;
     if (rest > n1) {
       chol::GemmProblem q{};  // rows below the next diagonal block, its columns
-      q.A = at(A, k1 + n1, k0); q.lda = di; q.B = at(A, k1, k0); q.ldb = di;
+      q.A = at(A, k1 + n1, ka); q.lda = di; q.B = at(A, k1, ka); q.ldb = di;
       q.C = at(A, k1 + n1, k1); q.ldc = di;
-      q.M = rest - n1; q.N = n1; q.K = nk; q.alpha = -1.0; q.beta = 1.0;
+      q.M = rest - n1; q.N = n1; q.K = kK; q.alpha = -1.0; q.beta = 1.0;
       uk.push_back(q);
-      chol::GemmProblem r{};  // the rest of the trailing matrix, lower tiles
-      r.A = at(A, k1 + n1, k0); r.lda = di; r.B = at(A, k1 + n1, k0); r.ldb = di;
-      r.C = at(A, k1 + n1, k1 + n1); r.ldc = di;
-      r.M = rest - n1; r.N = rest - n1; r.K = nk; r.lower_only = 1; r.alpha = -1.0; r.beta = 1.0;
-      uk.push_back(r);
-    }
-    if (k0 > 0) {
-      chol::GemmProblem q{};  // Mt[:k0, k1:] -= Mt[:k0, block k] L21^T
-      q.A = at(Mt, 0, k0); q.lda = di; q.B = at(A, k1, k0); q.ldb = di;
-      q.C = at(Mt, 0, k1); q.ldc = di;
-      q.M = k0; q.N = rest; q.K = nk; q.alpha = -1.0; q.beta = 1.0;
-      uk.push_back(q);
+      const int c2 = w1 - (k1 + n1);  // the further columns to update
+      if (c2 > 0) {
+        chol::GemmProblem r{};  // their square part, lower tiles
+        r.A = at(A, k1 + n1, ka); r.lda = di; r.B = at(A, k1 + n1, ka); r.ldb = di;
+        r.C = at(A, k1 + n1, k1 + n1); r.ldc = di;
+        r.M = c2; r.N = c2; r.K = kK; r.lower_only = 1; r.alpha = -1.0; r.beta = 1.0;
+        uk.push_back(r);
+        if (di > w1) {
+          chol::GemmProblem t{};  // the rows under the window's square part
+          t.A = at(A, w1, ka); t.lda = di; t.B = at(A, k1 + n1, ka); t.ldb = di;
+          t.C = at(A, w1, k1 + n1); t.ldc = di;
+          t.M = di - w1; t.N = c2; t.K = kK; t.alpha = -1.0; t.beta = 1.0;
+          uk.push_back(t);
+        }
+      }
     }
     {
-      chol::GemmProblem q{};  // Mt[block k, k1:] = -X_kk^T L21^T (first write)
-      q.A = at(Mt, k0, k0); q.lda = di; q.B = at(A, k1, k0); q.ldb = di;
-      q.C = at(Mt, k0, k1); q.ldc = di;
-      q.M = nk; q.N = rest; q.K = nk; q.alpha = -1.0; q.beta = 0.0;
+      chol::GemmProblem q{};  // Mt[:k1, k1:w1] -= Mt[:k1, ka:k1] L[k1:w1, ka:k1]^T
+      q.A = at(Mt, 0, ka); q.lda = di; q.B = at(A, k1, ka); q.ldb = di;
+      q.C = at(Mt, 0, k1); q.ldc = di;
+      q.M = k1; q.N = w1 - k1; q.K = kK; q.alpha = -1.0; q.beta = 1.0;
       uk.push_back(q);
     }
     // two SMs stay free for D_k and leaf k+1 on the auxiliary stream (the

@@ -168,7 +168,8 @@ def gptq_prepare_hinv(H: torch.Tensor, damp_rel: float, G: torch.Tensor,
                       stream=None) -> int:
     """G = upper U with U^T U = (H + damp)^-1.  Returns bad_pivot (-1 if SPD)."""
     d = H.shape[0]
-    assert G.dtype == torch.float32 and G.shape == (d, d)
+    assert H.dtype == torch.float32 and H.shape == (d, d) and H.is_contiguous()
+    assert G.dtype == torch.float32 and G.shape == (d, d) and G.is_contiguous()
     assert dead_mask.dtype == torch.uint8 and dead_mask.numel() == d
     piv = ctypes.c_int64(-1)
     st = load_library().gptq_prepare_hinv(
@@ -184,6 +185,7 @@ def gptq_quantize_layer(W: torch.Tensor, G: torch.Tensor, dead_mask,
                         ws: torch.Tensor, stream=None) -> None:
     d_row, d_col = W.shape
     assert W.dtype == torch.float32 and W.is_contiguous()
+    assert G.dtype == torch.float32 and G.shape == (d_col, d_col) and G.is_contiguous()
     assert qweight.dtype == torch.int32 or qweight.dtype == torch.uint32
     st = load_library().gptq_quantize_layer(
         _ptr(W), d_row, d_col, _ptr(G), _ptr(dead_mask), ctypes.byref(cfg),
