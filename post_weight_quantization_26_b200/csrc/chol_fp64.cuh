@@ -40,7 +40,7 @@ constexpr int NB = 128;  // panel / leaf width
 // Panels per lazy-update window (see gptq_prepare_hinv): the window's last
 // panel applies all of them to the trailing matrix at once (K = 128 m).
 #ifndef GPTQ_WINDOW_PANELS
-#define GPTQ_WINDOW_PANELS 4
+#define GPTQ_WINDOW_PANELS 8
 #endif
 inline int window_panels(int d) { return d >= 8192 ? GPTQ_WINDOW_PANELS : 1; }
 
@@ -439,7 +439,10 @@ leaf_kernel(const double* __restrict__ A, double* __restrict__ Mt, double* __res
 // slices of 16 along K are copied by cp.async (16-byte chunks, zero fill
 // outside the matrix) into [row][k] tiles padded to 20 doubles per row, so
 // both the copies and the fragment reads are free of bank conflicts.
-constexpr int TN = 128, TK = 16, LDS = TK + 4, GSTAGES = 3;
+#ifndef GPTQ_DGEMM_TK
+#define GPTQ_DGEMM_TK 32
+#endif
+constexpr int TN = 128, TK = GPTQ_DGEMM_TK, LDS = TK + 4, GSTAGES = 3;
 constexpr int MAXP = 64;
 
 struct GemmProblem {

@@ -182,16 +182,18 @@ PrepareWs prepare_layout(int64_t d) {
 }
 
 struct QuantWs {
-  size_t Wk, E[2][2], Ghi, Glo, total;  // E[buffer][hi/lo]
+  size_t Wk, E[2][2], Ghi, Glo, total;  // E[window buffer][hi/lo]
+  int lde;                              // E row stride: one window of blocks
 };
 QuantWs quant_layout(int64_t d_row, int64_t d_col, int block) {
   QuantWs w{};
+  w.lde = quant::sweep_window_blocks(d_col) * block;
   size_t off = 0;
   w.Wk = off; off = align_up(off + static_cast<size_t>(d_row) * d_col * 4);
   for (int b = 0; b < 2; ++b)
     for (int h = 0; h < 2; ++h) {
       w.E[b][h] = off;
-      off = align_up(off + static_cast<size_t>(d_row) * block * 4);
+      off = align_up(off + static_cast<size_t>(d_row) * w.lde * 4);
     }
   w.Ghi = off; off = align_up(off + static_cast<size_t>(d_col) * d_col * 4);
   w.Glo = off; off = align_up(off + static_cast<size_t>(d_col) * d_col * 4);
@@ -766,11 +768,13 @@ gptq_status gptq_quantize_layer(const float* W, int64_t d_row, int64_t d_col, co
   int num_sms = 148;
   st = device_setup(&num_sms);
   if (st != GPTQ_OK) return st;
-  // tensor maps of the trailing update: E splits (K-major), G splits, W
+  // tensor maps of the trailing update: E splits (K-major, one window of
+  // blocks per row), G splits, W
+  const int lde = L.lde, mw = lde / B;
   CUtensorMap tm_e[2][2], tm_ghi, tm_glo, tm_w;
   for (int b = 0; b < 2; ++b)
     for (int h = 0; h < 2; ++h) {
-      st = encode_f32_2d(&tm_e[b][h], Eb[b][h], B, dr, B, trail::BK, trail::BM,
+      st = encode_f32_2d(&tm_e[b][h], Eb[b][h], lde, dr, lde, trail::BK, trail::BM,
                          CU_TENSOR_MAP_SWIZZLE_64B);
       if (st != GPTQ_OK) return st;
     }
@@ -791,8 +795,12 @@ gptq_status gptq_quantize_layer(const float* W, int64_t d_row, int64_t d_col, co
   // Block j: the step kernel Q_j (caller's stream) applies E_{j-1} to block j
   // and quantizes it; the trailing kernel T_j (auxiliary stream) applies E_j
   // to the columns right of block j+1.  Q_j needs T_{j-2} (it finished
-  // block j's earlier updates; also frees E buffer j%2); T_j needs Q_j.  So
-  // Q_{j+1} overlaps T_j.
+  // block j's earlier updates); T_j needs Q_j.  So Q_{j+1} overlaps T_j.
+  // The updates are lazy over windows of mw blocks: inside a window, T_j
+  // reaches only the window's remaining columns; the window's last block
+  // applies all the window's errors (K = mw B) to everything right of the
+  // next block, and the next window's first step applies them to itself.
+  // The errors of a window stay in one of two E buffers (row stride lde).
   std::lock_guard<std::mutex> lk(di->qmu);
   cudaEvent_t ev_fork = di->ev[0], ev_join = di->ev[1];
   cudaEvent_t* evQ = di->ev + 2;
@@ -801,19 +809,44 @@ gptq_status gptq_quantize_layer(const float* W, int64_t d_row, int64_t d_col, co
   GPTQ_CUDA_TRY(cudaStreamWaitEvent(di->aux, ev_fork, 0));
   const int nblk = (dc + B - 1) / B;
   const dim3 qgrid((dr + quant::QROWS - 1) / quant::QROWS);
-  std::vector<char> t_done(nblk, 0);
+  // W[:, n0:n1] -= E[buf][:, ek0:ek0+K] * G[gj0:gj0+K, n0:n1]
+  auto trailing = [&](int buf, int ek0, int K, int gj0, int n0, int n1) -> gptq_status {
+    trail::Params tp{};
+    tp.M = dr; tp.N = n1 - n0; tp.K = K; tp.n0 = n0; tp.j0 = gj0; tp.ek0 = ek0;
+    tp.chain = 256 / trail::BK;  // a window's update is summed 256 columns at a time
+    tp.wait_ns = g_wait_ns.load();
+    tp.stall = g_fault.load() == GPTQ_FAULT_TRAILING_STALL;
+    tp.tiles_m = (dr + trail::BM - 1) / trail::BM;
+    tp.tiles_n = (tp.N + trail::BN - 1) / trail::BN;
+    tp.tiles = tp.tiles_m * tp.tiles_n;
+    const int grid = std::min(tp.tiles, num_sms);
+    trail::trailing_tf32x3_kernel<<<grid, trail::NUM_THREADS, trail::SMEM_BYTES, di->aux>>>(
+        tm_e[buf][0], tm_e[buf][1], tm_ghi, tm_glo, tm_w, tp);
+    GPTQ_LAUNCH_CHECK();
+    return GPTQ_OK;
+  };
   for (int jb = 0; jb < nblk; ++jb) {
     const int j0 = jb * B, ncols = std::min(B, dc - j0);
-    if (jb >= 2 && t_done[jb - 2]) GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, evT[(jb - 2) % 4], 0));
-    if (g > B && j0 % g == 0 && jb >= 1 && t_done[jb - 1])  // group params read columns ahead
+    const int win = jb / mw, pos = jb % mw, e0 = win * mw * B, e1 = std::min(dc, e0 + mw * B);
+    const int cb = win & 1, pb = (win - 1) & 1;
+    if (jb >= 2) GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, evT[(jb - 2) % 4], 0));
+    if (g > B && j0 % g == 0 && jb >= 1)  // group params read columns ahead
       GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, evT[(jb - 1) % 4], 0));
-    const int pb = (jb - 1) & 1, cb = jb & 1;
-    const float* Eph = jb > 0 ? Eb[pb][0] : nullptr;
-    const float* Epl = jb > 0 ? Eb[pb][1] : nullptr;
-    const int jp0 = jb > 0 ? j0 - B : -1;
+    // the previous block, or at a window's first block the whole previous window
+    const float *Eph = nullptr, *Epl = nullptr;
+    int jp0 = -1, nprev = 0;
+    if (jb > 0 && pos > 0) {
+      Eph = Eb[cb][0] + (pos - 1) * B; Epl = Eb[cb][1] + (pos - 1) * B;
+      jp0 = j0 - B; nprev = B;
+    } else if (jb > 0) {
+      Eph = Eb[pb][0]; Epl = Eb[pb][1];
+      jp0 = e0 - mw * B; nprev = mw * B;
+    }
+    float* Ech = Eb[cb][0] + pos * B;
+    float* Ecl = Eb[cb][1] + pos * B;
 #define GPTQ_STEP(BB)                                                                        \
   quant::block_step_kernel<BB><<<qgrid, quant::QTHREADS, quant::block_step_smem<BB>(), s>>>( \
-      Wk, dr, dc, j0, ncols, G, Eph, Epl, jp0, Eb[cb][0], Eb[cb][1], qweight, scales, zeros,   \
+      Wk, dr, dc, j0, ncols, G, Eph, Epl, jp0, nprev, lde, Ech, Ecl, qweight, scales, zeros,  \
       cfg->bits, cfg->sym, g, n_groups, per_channel)
     if (B == 128) GPTQ_STEP(128);
     else if (B == 64) GPTQ_STEP(64);
@@ -821,23 +854,18 @@ gptq_status gptq_quantize_layer(const float* W, int64_t d_row, int64_t d_col, co
 #undef GPTQ_STEP
     GPTQ_LAUNCH_CHECK();
     GPTQ_CUDA_TRY(cudaEventRecord(evQ[jb % 4], s));
-    const int n0 = j0 + 2 * B;  // block jb+1 is updated by Q_{jb+1} itself
-    if (n0 < dc) {
-      GPTQ_CUDA_TRY(cudaStreamWaitEvent(di->aux, evQ[jb % 4], 0));
-      trail::Params tp{};
-      tp.M = dr; tp.N = dc - n0; tp.K = ncols; tp.n0 = n0; tp.j0 = j0;
-      tp.wait_ns = g_wait_ns.load();
-      tp.stall = g_fault.load() == GPTQ_FAULT_TRAILING_STALL;
-      tp.tiles_m = (dr + trail::BM - 1) / trail::BM;
-      tp.tiles_n = (tp.N + trail::BN - 1) / trail::BN;
-      tp.tiles = tp.tiles_m * tp.tiles_n;
-      const int grid = std::min(tp.tiles, num_sms);
-      trail::trailing_tf32x3_kernel<<<grid, trail::NUM_THREADS, trail::SMEM_BYTES, di->aux>>>(
-          tm_e[cb][0], tm_e[cb][1], tm_ghi, tm_glo, tm_w, tp);
-      GPTQ_LAUNCH_CHECK();
-      GPTQ_CUDA_TRY(cudaEventRecord(evT[jb % 4], di->aux));
-      t_done[jb] = 1;
+    GPTQ_CUDA_TRY(cudaStreamWaitEvent(di->aux, evQ[jb % 4], 0));
+    if (pos < mw - 1 && j0 + ncols < dc) {
+      // inside the window: this block's errors on the window's remaining
+      // columns (block jb+1 takes them in its own step)
+      if (e1 > j0 + 2 * B && (st = trailing(cb, pos * B, ncols, j0, j0 + 2 * B, e1)) != GPTQ_OK)
+        return st;
+    } else if (e1 + B < dc) {
+      // the window's last block: all its errors on everything right of the
+      // next block (which takes them in its own step)
+      if ((st = trailing(cb, 0, e1 - e0, e0, e1 + B, dc)) != GPTQ_OK) return st;
     }
+    GPTQ_CUDA_TRY(cudaEventRecord(evT[jb % 4], di->aux));
   }
   GPTQ_CUDA_TRY(cudaEventRecord(ev_join, di->aux));
   GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, ev_join, 0));

@@ -5,7 +5,8 @@
 //
 // Per block j0 (block_step_kernel, one CTA per 32 rows):
 //   (a) apply the previous block's errors to this block, W -= E_prev G
-//       (m16n8k8 tf32 MMAs on the split operands);
+//       (m16n8k8 tf32 MMAs on the split operands); at the first block of a
+//       lazy-update window, the errors of the whole previous window;
 //   (b) the B columns of every row: parameters at a group start, code,
 //       dequantize, e = (w - w^)/G_qq, subtract e * G[q, k] from the later
 //       columns of the block, keep e in E.  A row's values live in
@@ -114,6 +115,17 @@ __global__ void prepare_rows_kernel(const float* __restrict__ W, float* __restri
 constexpr int QROWS = 32;            // rows per CTA
 constexpr int QTHREADS = QROWS * 4;  // 4 threads per row
 
+// Blocks per lazy-update window of the sweep (see gptq_quantize_layer): the
+// trailing update after each block touches only the window's remaining
+// columns, and the window's last block updates everything to the right of
+// the next block with all m blocks at once (K = m B).  Wide layers only: it
+// cuts the trailing read-modify-write traffic on W by m, which is what
+// bounds the sweep there.
+#ifndef GPTQ_SWEEP_WINDOW
+#define GPTQ_SWEEP_WINDOW 4
+#endif
+inline int sweep_window_blocks(int64_t d_col) { return d_col >= 8192 ? GPTQ_SWEEP_WINDOW : 1; }
+
 template <int B>
 struct StepSmem {
   static constexpr int LDG = B + 4;  // padded rows (floats)
@@ -182,10 +194,11 @@ template <int B>
 __global__ void __launch_bounds__(QTHREADS)
 block_step_kernel(const float* __restrict__ Wk, int d_row, int d_col, int j0, int ncols,
                   const float* __restrict__ G, const float* __restrict__ Eprev_hi,
-                  const float* __restrict__ Eprev_lo, int jp0, float* __restrict__ Ecur_hi,
-                  float* __restrict__ Ecur_lo, uint32_t* __restrict__ qweight,
-                  float* __restrict__ scales, uint8_t* __restrict__ zeros, int bits, int sym,
-                  int group, int n_groups, int pc_mode) {
+                  const float* __restrict__ Eprev_lo, int jp0, int nprev, int lde,
+                  float* __restrict__ Ecur_hi, float* __restrict__ Ecur_lo,
+                  uint32_t* __restrict__ qweight, float* __restrict__ scales,
+                  uint8_t* __restrict__ zeros, int bits, int sym, int group, int n_groups,
+                  int pc_mode) {
   using L = StepSmem<B>;
   constexpr int LDG = L::LDG;
   extern __shared__ __align__(16) uint8_t qsm[];
@@ -202,55 +215,77 @@ block_step_kernel(const float* __restrict__ Wk, int d_row, int d_col, int j0, in
   const int r = r0 + rloc;
   const bool rv = r < d_row;
 
+  // E_prev (nprev columns, row stride lde) and the G rows [jp0, jp0 + nprev)
+  // are taken in chunks of B columns
+  auto stage_chunk = [&](int kc) {
+    stage_rows<B>(Es, Eprev_hi + kc, lde, r0, d_row, B, tid);
+    stage_gblock<B>(Gs, G, d_col, jp0 + kc, j0, B, ncols, tid);
+  };
   stage_rows<B>(Ws, Wk + j0, d_col, r0, d_row, ncols, tid);
-  if (jp0 >= 0) {
-    stage_rows<B>(Es, Eprev_hi, B, r0, d_row, B, tid);
-    stage_gblock<B>(Gs, G, d_col, jp0, j0, B, ncols, tid);
-  } else {
-    stage_gblock<B>(Gs, G, d_col, j0, j0, ncols, ncols, tid);
-  }
+  if (nprev > 0) stage_chunk(0);
+  else stage_gblock<B>(Gs, G, d_col, j0, j0, ncols, ncols, tid);
   asm volatile("cp.async.commit_group;" ::: "memory");
   asm volatile("cp.async.wait_group 0;" ::: "memory");
   __syncthreads();
-  if (jp0 >= 0) {  // E = E_hi + E_lo (exact): add the low parts in place
-    for (int c = tid; c < QROWS * (B / 4); c += QTHREADS) {
-      const int rr = c / (B / 4), k = (c - rr * (B / 4)) * 4;
-      if (r0 + rr < d_row) {
-        const float4 lo = *reinterpret_cast<const float4*>(Eprev_lo + static_cast<size_t>(r0 + rr) * B + k);
-        float4* hp = reinterpret_cast<float4*>(Es + rr * L::LDG + k);
-        float4 h = *hp;
-        h.x += lo.x; h.y += lo.y; h.z += lo.z; h.w += lo.w;
-        *hp = h;
-      }
-    }
-    __syncthreads();
-  }
 
   float* wrow = Ws + rloc * LDG;
   float* erow = Es + rloc * LDG;
-  if (jp0 >= 0) {
-    // (a) W[rows, blk] -= E_prev[rows] * G[prev blk, blk] on the MMA path:
+  if (nprev > 0) {
+    // (a) W[rows, blk] -= E_prev[rows] * G[prev cols, blk] on the MMA path:
     // m16n8k8 tf32, three products of the split operands (hi hi + hi lo +
     // lo hi; hi = the low 13 mantissa bits cleared), fp32 accumulate, the
-    // same arithmetic as the trailing update.  Warp w takes the output
-    // columns [w B/4, (w+1) B/4) of both 16-row halves of the slab; ncols is
-    // a multiple of 32, so a warp's columns are all inside or all past it.
-    {
-      constexpr int NTW = B / 32;  // 8-column tiles per warp
-      const int warp = tid >> 5, g = lane >> 2, t4 = lane & 3;
-      const int cw = warp * (B / 4);
+    // same arithmetic as the trailing update.  The previous columns are the
+    // previous block, or at a window's first block all the blocks of the
+    // previous window, B at a time.  Warp w takes the output columns
+    // [w B/4, (w+1) B/4) of both 16-row halves of the slab; ncols is a
+    // multiple of 32, so a warp's columns are all inside or all past it.
+    constexpr int NTW = B / 32;  // 8-column tiles per warp
+    const int warp = tid >> 5, g = lane >> 2, t4 = lane & 3;
+    const int cw = warp * (B / 4);
+    float acc[2][NTW][4];
+    if (cw < ncols) {
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < NTW; ++nt) {
+          const float* w0 = Ws + (16 * mt + g) * LDG + cw + 8 * nt + 2 * t4;
+          acc[mt][nt][0] = w0[0];
+          acc[mt][nt][1] = w0[1];
+          acc[mt][nt][2] = w0[8 * LDG];
+          acc[mt][nt][3] = w0[8 * LDG + 1];
+        }
+    }
+    // each chunk of B columns is summed from zero and then added into the
+    // block with round-to-nearest fp32 adds: the MMA's own accumulation does
+    // not round to nearest, and its error grows with the MMAs it chains
+    float part[2][NTW][4];
+    for (int kc = 0; kc < nprev; kc += B) {
+      if (kc > 0) {
+        stage_chunk(kc);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        __syncthreads();
+      }
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < NTW; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) part[mt][nt][e] = 0.0f;
+      // E = E_hi + E_lo (exact): add the low parts in place
+      for (int c = tid; c < QROWS * (B / 4); c += QTHREADS) {
+        const int rr = c / (B / 4), k = (c - rr * (B / 4)) * 4;
+        if (r0 + rr < d_row) {
+          const float4 lo = *reinterpret_cast<const float4*>(
+              Eprev_lo + static_cast<size_t>(r0 + rr) * lde + kc + k);
+          float4* hp = reinterpret_cast<float4*>(Es + rr * L::LDG + k);
+          float4 h = *hp;
+          h.x += lo.x; h.y += lo.y; h.z += lo.z; h.w += lo.w;
+          *hp = h;
+        }
+      }
+      __syncthreads();
       if (cw < ncols) {
-        float acc[2][NTW][4];
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-          for (int nt = 0; nt < NTW; ++nt) {
-            const float* w0 = Ws + (16 * mt + g) * LDG + cw + 8 * nt + 2 * t4;
-            acc[mt][nt][0] = w0[0];
-            acc[mt][nt][1] = w0[1];
-            acc[mt][nt][2] = w0[8 * LDG];
-            acc[mt][nt][3] = w0[8 * LDG + 1];
-          }
 #pragma unroll 2
         for (int k0 = 0; k0 < B; k0 += 8) {
           uint32_t ah[2][4], al[2][4];
@@ -269,25 +304,33 @@ block_step_kernel(const float* __restrict__ Wk, int d_row, int d_col, int j0, in
             split_tf32(g0[4 * LDG], bh1, bl1);
 #pragma unroll
             for (int mt = 0; mt < 2; ++mt) {
-              mma_tf32_m16n8k8(acc[mt][nt], ah[mt], bh0, bh1);
-              mma_tf32_m16n8k8(acc[mt][nt], ah[mt], bl0, bl1);
-              mma_tf32_m16n8k8(acc[mt][nt], al[mt], bh0, bh1);
+              mma_tf32_m16n8k8(part[mt][nt], ah[mt], bh0, bh1);
+              mma_tf32_m16n8k8(part[mt][nt], ah[mt], bl0, bl1);
+              mma_tf32_m16n8k8(part[mt][nt], al[mt], bh0, bh1);
             }
           }
         }
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-          for (int nt = 0; nt < NTW; ++nt) {
-            float* w0 = Ws + (16 * mt + g) * LDG + cw + 8 * nt + 2 * t4;
-            w0[0] = acc[mt][nt][0];
-            w0[1] = acc[mt][nt][1];
-            w0[8 * LDG] = acc[mt][nt][2];
-            w0[8 * LDG + 1] = acc[mt][nt][3];
-          }
+          for (int nt = 0; nt < NTW; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[mt][nt][e] += part[mt][nt][e];
       }
+      __syncthreads();  // every thread is done with this chunk's E and G rows
     }
-    __syncthreads();  // every thread is done with the previous block's G rows
+    if (cw < ncols) {
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < NTW; ++nt) {
+          float* w0 = Ws + (16 * mt + g) * LDG + cw + 8 * nt + 2 * t4;
+          w0[0] = acc[mt][nt][0];
+          w0[1] = acc[mt][nt][1];
+          w0[8 * LDG] = acc[mt][nt][2];
+          w0[8 * LDG + 1] = acc[mt][nt][3];
+        }
+    }
     stage_gblock<B>(Gs, G, d_col, j0, j0, ncols, ncols, tid);
     asm volatile("cp.async.commit_group;" ::: "memory");
     asm volatile("cp.async.wait_group 0;" ::: "memory");
@@ -390,8 +433,8 @@ block_step_kernel(const float* __restrict__ Wk, int d_row, int d_col, int j0, in
   // (c) E for the trailing update as a TF32 split (hi = low 13 mantissa bits
   // cleared, lo = E - hi), and the packed codes
   if (rv) {
-    float* eh = Ecur_hi + static_cast<size_t>(r) * B;
-    float* el = Ecur_lo + static_cast<size_t>(r) * B;
+    float* eh = Ecur_hi + static_cast<size_t>(r) * lde;
+    float* el = Ecur_lo + static_cast<size_t>(r) * lde;
     for (int c = 4 * t; c < B; c += 16) {
       const float4 v = (c < ncols) ? *reinterpret_cast<const float4*>(erow + c)
                                    : make_float4(0.f, 0.f, 0.f, 0.f);

@@ -2,7 +2,7 @@
 // tensor cores (dingiv.github.io "量化" page, section GPTQ: after a block of B
 // columns is quantized, all columns to its right are updated at once by one
 // matrix product):
-//     W[:, n0:] -= E * G[j0:j0+K, n0:]
+//     W[:, n0:n0+N] -= E[:, ek0:ek0+K] * G[j0:j0+K, n0:n0+N]
 // E (d_row x K) and G are fp32; the product runs as three TF32 MMAs per
 // K-step on the split operands x = x_hi + x_lo (x_hi = x with the low 13
 // mantissa bits cleared, x_lo = x - x_hi, exact):
@@ -22,7 +22,8 @@
 //   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, negate, write a
 //               128x32 tile to shared memory (128-byte swizzle), and add it
 //               into W with a TMA reduce-add (the L2 does the read-modify-
-//               write).
+//               write).  A long K is summed in chains of `chain` K-steps,
+//               each added into W on its own, in order.
 // Shared memory is kept near 112 KB so a block-step CTA fits on the same SM
 // (the two kernels run concurrently on different streams).  Every mbarrier
 // wait is bounded.
@@ -57,6 +58,8 @@ struct Params {
   int K;        // block width (E and G read as zero past it)
   int n0;       // first column to update (also the column coordinate into G)
   int j0;       // first row of G's block
+  int ek0;      // first column of E's block in the E buffer
+  int chain;    // K-steps (of BK) summed per TMEM chain; 0: the whole K in one
   int tiles_m, tiles_n, tiles;
   uint64_t wait_ns;  // limit of every bounded wait (ns)
   int stall;    // fault injection: the producer issues nothing, so the MMA
@@ -125,6 +128,10 @@ trailing_tf32x3_kernel(const __grid_constant__ CUtensorMap tm_ehi,
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int nk = (p.K + BK - 1) / BK;  // E is zero past K
+  // K-steps per TMEM chain: each chain is summed from zero and added into W
+  // on its own (round-to-nearest in L2), since the MMA's accumulation does
+  // not round to nearest and its error grows with the MMAs it chains
+  const int chain = p.chain > 0 ? p.chain : nk;
 
   if (warp == 0) {
     if (lane == 0 && !p.stall) {  // -------------------------------- producer
@@ -137,8 +144,8 @@ trailing_tf32x3_kernel(const __grid_constant__ CUtensorMap tm_ehi,
           const uint32_t fb = full0 + 8u * stage;
           mbar_arrive_expect_tx(fb, STAGE_BYTES);
           const uint32_t s0 = ring + stage * STAGE_BYTES;
-          tma_load_2d(s0, &tm_ehi, fb, ks * BK, tm * BM);
-          tma_load_2d(s0 + A_BYTES, &tm_elo, fb, ks * BK, tm * BM);
+          tma_load_2d(s0, &tm_ehi, fb, p.ek0 + ks * BK, tm * BM);
+          tma_load_2d(s0 + A_BYTES, &tm_elo, fb, p.ek0 + ks * BK, tm * BM);
           const int gx = p.n0 + tn * BN, gy = p.j0 + ks * BK;
 #pragma unroll
           for (int c = 0; c < BN / B_BOX; ++c) {
@@ -153,14 +160,18 @@ trailing_tf32x3_kernel(const __grid_constant__ CUtensorMap tm_ehi,
   } else if (warp == 1) {
     if (lane == 0) {  // ----------------------------------------------- MMA
       uint32_t stage = 0, phase = 0;
-      int lu = 0;
+      int lu = 0;  // chains issued by this CTA
       bool ok = true;
-      for (int u = blockIdx.x; u < p.tiles && ok; u += gridDim.x, ++lu) {
+      for (int u = blockIdx.x; u < p.tiles && ok; u += gridDim.x) {
+       for (int c0 = 0; c0 < nk && ok; c0 += chain, ++lu) {
         const uint32_t acc = lu & 1;
-        if (!mbar_wait_bounded(tempty0 + 8u * acc, ((lu >> 1) & 1) ^ 1u, abort_flag, p.wait_ns)) break;
+        if (!mbar_wait_bounded(tempty0 + 8u * acc, ((lu >> 1) & 1) ^ 1u, abort_flag, p.wait_ns)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
-        for (int ks = 0; ks < nk; ++ks) {
+        for (int ks = c0; ks < min(nk, c0 + chain); ++ks) {
           if (!mbar_wait_bounded(full0 + 8u * stage, phase, abort_flag, p.wait_ns)) { ok = false; break; }
           tc_fence_after();
           const uint32_t s0 = ring + stage * STAGE_BYTES;
@@ -175,7 +186,7 @@ trailing_tf32x3_kernel(const __grid_constant__ CUtensorMap tm_ehi,
             // are the kk-th 1 KB slice.
             const uint64_t bhi = smem_desc(s0 + 2 * A_BYTES + kk * 1024, B_BOX_BYTES, 512, 1);
             const uint64_t blo = smem_desc(s0 + 2 * A_BYTES + B_BYTES + kk * 1024, B_BOX_BYTES, 512, 1);
-            mma_tf32_ss(d_tmem, ahi, bhi, IDESC, (ks | kk) != 0);
+            mma_tf32_ss(d_tmem, ahi, bhi, IDESC, ((ks - c0) | kk) != 0);
             mma_tf32_ss(d_tmem, ahi, blo, IDESC, 1);
             mma_tf32_ss(d_tmem, alo, bhi, IDESC, 1);
           }
@@ -184,6 +195,7 @@ trailing_tf32x3_kernel(const __grid_constant__ CUtensorMap tm_ehi,
         }
         if (!ok) break;
         mma_commit(tfull0 + 8u * acc);
+       }
       }
     }
     __syncwarp();
@@ -197,11 +209,14 @@ trailing_tf32x3_kernel(const __grid_constant__ CUtensorMap tm_ehi,
     // waiting at a barrier it will not reach.
     bool ok = true;
     int lu = 0;
-    for (int u = blockIdx.x; u < p.tiles; u += gridDim.x, ++lu) {
-      const int tm = u % p.tiles_m, tn = u / p.tiles_m;
+    for (int u = blockIdx.x; u < p.tiles; u += gridDim.x) {
+     const int tm = u % p.tiles_m, tn = u / p.tiles_m;
+     for (int c0 = 0; c0 < nk; c0 += chain, ++lu) {
       const uint32_t acc = lu & 1;
       if (ok && !mbar_wait_bounded(tfull0 + 8u * acc, (lu >> 1) & 1, abort_flag, p.wait_ns)) ok = false;
       tc_fence_after();
+      // a tile's chains land in W in order: the previous chain's adds first
+      if (issuer && c0 > 0) bulk_wait0();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
       for (int c = 0; c < BN / OUT_COLS; ++c) {
         if (p.n0 + tn * BN + c * OUT_COLS >= p.n0 + p.N) break;  // past the matrix
@@ -234,6 +249,7 @@ trailing_tf32x3_kernel(const __grid_constant__ CUtensorMap tm_ehi,
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty0 + 8u * acc);
+     }
     }
     if (issuer) bulk_wait0();
   }

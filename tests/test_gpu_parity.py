@@ -194,6 +194,35 @@ def test_quantize_matches_oracle(G, case):
     check_layer(codes, sc, ze, ref_codes, ref_s, ref_z, group)
 
 
+_WIDE = {}
+
+
+def _wide_factor(d_col):
+    """The oracle's fp32-rounded factor for a wide test layer (computed once)."""
+    if d_col not in _WIDE:
+        spec = synth.tiny_spec(8, d_col, d_col + 512, seed=d_col)
+        hd, _ = O.dampen(O.hessian(synth.gen_tokens(spec).float().numpy()), 0.01)
+        _WIDE[d_col] = np.ascontiguousarray(O.hinv_cholesky_upper(hd), dtype=np.float32)
+    return _WIDE[d_col]
+
+
+@pytest.mark.parametrize("case", [(48, 8448, 4, 128, False, 128), (40, 8448, 3, 0, False, 64),
+                                  (24, 8448, 4, 256, True, 128)],
+                         ids=lambda c: "x".join(map(str, c)))
+def test_quantize_wide_layers_lazy_windows(G, case):
+    """Layers of 8192 columns or more sweep in lazy-update windows of blocks
+    (the errors of a window reach the columns right of it at once, and the
+    next window's first block takes them in its own step); here the last
+    window is partial (66 or 132 blocks) and g = 256 spans two blocks."""
+    d_row, d_col, bits, group, sym, block = case
+    w = synth.gen_weight(synth.tiny_spec(d_row, d_col, 8, seed=d_row + bits)).numpy()
+    u32 = _wide_factor(d_col)
+    codes, sc, ze, _ = _run_quantize(G, w, u32, bits, group, sym, block)
+    ref_codes, ref_s, ref_z, _, _ = O.gptq_quantize(
+        w.astype(np.float64), u32.astype(np.float64), bits, group, sym, block)
+    check_layer(codes, sc, ze, ref_codes, ref_s, ref_z, group)
+
+
 def test_quantize_scaled_identity_is_rtn(G):
     """With G = c I nothing propagates: GPU output equals round-to-nearest."""
     spec = synth.tiny_spec(64, 256, 16)
