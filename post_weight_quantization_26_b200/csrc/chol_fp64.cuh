@@ -23,7 +23,7 @@
 // inside a window U_k and D_k apply panel k only to the window's remaining
 // columns; the window's last panel applies all m panels (K = 128 m) to
 // everything right of the window.  Same sums, regrouped, so most of the
-// 2/3 d^3 flops run with a 4x longer K per output tile and a quarter of the
+// 2/3 d^3 flops run with an m times longer K per output tile and 1/m of the
 // trailing matrix's read-modify-write traffic.
 // Every product is an "NT" GEMM (both operands row-major along K) on the
 // fp64 MMA path (mma.sync m8n8k4 f64), staged by cp.async through a 3-deep
@@ -434,11 +434,15 @@ leaf_kernel(const double* __restrict__ A, double* __restrict__ Mt, double* __res
 
 // ------------------------------------------------------------ NT DGEMM
 // C[m][n] = alpha * sum_k A[m][k] B[n][k] + beta * C[m][n]  for up to MAXP
-// problems per launch.  TM x 128 tile per CTA, NW warps in a WGM x (NW/WGM)
-// grid, each warp an (MI*8) x (NI*8) block of m8n8k4 fp64 MMAs.  A and B
-// slices of 16 along K are copied by cp.async (16-byte chunks, zero fill
-// outside the matrix) into [row][k] tiles padded to 20 doubles per row, so
-// both the copies and the fragment reads are free of bank conflicts.
+// problems per launch.  A CTA holds NG independent warp groups; each group
+// runs its own persistent loop over TM x TNG tiles with NW warps in a
+// WGM x (NW/WGM) grid (each warp an (MI*8) x (NI*8) block of m8n8k4 fp64
+// MMAs), its own STG-deep ring of shared-memory stages and its own named
+// barrier, so one group's epilogue and slice barriers overlap the other
+// group's MMAs.  A and B slices of TKG along K are copied by cp.async
+// (16-byte chunks, zero fill outside the matrix) into [row][k] tiles padded
+// to TKG + 4 doubles per row, so both the copies and the fragment reads are
+// free of bank conflicts.
 #ifndef GPTQ_DGEMM_TK
 #define GPTQ_DGEMM_TK 32
 #endif
@@ -461,32 +465,52 @@ struct GemmBatch {
   GemmProblem p[MAXP];
 };
 
-template <int TM>
+template <int TM, int TNG = TN, int NG = 1, int TKG = TK, int STG = GSTAGES>
 constexpr int gemm_smem() {
-  return GSTAGES * (TM + TN) * LDS * 8;
+  return NG * STG * (TM + TNG) * (TKG + 4) * 8;
 }
 
+// Tiles of a lower_only (square) problem: those whose first column is on
+// or left of the tile row's last row, tile_n * TNG <= (tile_m + 1) TM - 1.
+// (The kernel decodes this order for TM == TNG and TM == 2 TNG, the shapes
+// that lower_only problems are launched with.)
+template <int TM, int TNG>
+inline int lower_tiles(int M, int N) {
+  const int tm = (M + TM - 1) / TM, tn = (N + TNG - 1) / TNG;
+  int n = 0;
+  for (int r = 0; r < tm; ++r) {
+    const int c = ((r + 1) * TM - 1) / TNG + 1;
+    n += c < tn ? c : tn;
+  }
+  return n;
+}
 
-
-// NW warps (NW * 32 threads) in a WGM x (NW / WGM) grid.
-template <int TM, int WGM, int NW = 8>
-__global__ void __launch_bounds__(NW * 32, 1)
+// NW warps per group (NW * 32 threads) in a WGM x (NW / WGM) grid.
+template <int TM, int WGM, int NW = 8, int TNG = TN, int NG = 1, int TKG = TK,
+          int STG = GSTAGES>
+__global__ void __launch_bounds__(NG * NW * 32, 1)
 dgemm_nt_kernel(const __grid_constant__ GemmBatch batch) {
-  constexpr int NTHREADS = NW * 32;
+  constexpr int NTHREADS = NW * 32;  // threads per group
+  constexpr int LDS = TKG + 4;       // padded stage row (doubles)
   constexpr int WGN = NW / WGM;
-  constexpr int WM = TM / WGM, WN = TN / WGN;
+  constexpr int WM = TM / WGM, WN = TNG / WGN;
   constexpr int MI = WM / 8, NI = WN / 8;
   extern __shared__ __align__(16) double gsm[];
-  double* As = gsm;                              // GSTAGES x TM x LDS
-  double* Bs = gsm + GSTAGES * TM * LDS;         // GSTAGES x TN x LDS
+  const int grp = NG > 1 ? static_cast<int>(threadIdx.x) / NTHREADS : 0;
+  double* As = gsm + grp * STG * (TM + TNG) * LDS;   // STG x TM x LDS
+  double* Bs = As + STG * TM * LDS;                   // STG x TNG x LDS
+  auto group_sync = [&]() {
+    if (NG == 1) __syncthreads();
+    else named_bar(1 + grp, NTHREADS);
+  };
 
-  const int bid = blockIdx.x;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = static_cast<int>(threadIdx.x) - grp * NTHREADS, lane = tid & 31, warp = tid >> 5;
   const int wm = warp / WGN, wn = warp % WGN;
   const int total = batch.tile_start[batch.count];
-  // Static persistent schedule: CTA c takes tiles c, c + grid, ...
-  int t = bid;
-  const int step = static_cast<int>(gridDim.x);
+  // Static persistent schedule: group g of CTA c takes tiles c NG + g, then
+  // every NG * grid-th tile after it
+  int t = static_cast<int>(blockIdx.x) * NG + grp;
+  const int step = static_cast<int>(gridDim.x) * NG;
 
   // A tile's problem lives in registers (the batch is only read here, once
   // per tile: fields read through a pointer into the parameter block would
@@ -505,14 +529,20 @@ dgemm_nt_kernel(const __grid_constant__ GemmBatch batch) {
     const GemmProblem& q = batch.p[pi];
     const int lt = tt - batch.tile_start[pi];
     int tm_i, tn_i;
-    if (q.lower_only) {
+    if (q.lower_only && TM == TNG) {  // row r holds r + 1 tiles
       int rr = static_cast<int>((sqrt(8.0 * lt + 1.0) - 1.0) * 0.5);
       while ((rr + 1) * (rr + 2) / 2 <= lt) ++rr;
       while (rr * (rr + 1) / 2 > lt) --rr;
       tm_i = rr;
       tn_i = lt - rr * (rr + 1) / 2;
+    } else if (q.lower_only && TM == 2 * TNG) {  // row r holds 2r + 2 tiles (the last may hold fewer)
+      int rr = static_cast<int>((sqrt(4.0 * lt + 1.0) - 1.0) * 0.5);
+      while ((rr + 1) * (rr + 2) <= lt) ++rr;
+      while (rr * (rr + 1) > lt) --rr;
+      tm_i = rr;
+      tn_i = lt - rr * (rr + 1);
     } else {
-      const int tn = (q.N + TN - 1) / TN;
+      const int tn = (q.N + TNG - 1) / TNG;
       tm_i = lt / tn;
       tn_i = lt - tm_i * tn;
     }
@@ -521,22 +551,22 @@ dgemm_nt_kernel(const __grid_constant__ GemmBatch batch) {
     T.lda = q.lda; T.ldb = q.ldb; T.ldc = q.ldc;
     T.M = q.M; T.N = q.N; T.K = q.K;
     T.alpha = q.alpha; T.beta = q.beta;
-    T.m0 = tm_i * TM; T.n0 = tn_i * TN; T.ns = (q.K + TK - 1) / TK;
+    T.m0 = tm_i * TM; T.n0 = tn_i * TNG; T.ns = (q.K + TKG - 1) / TKG;
     return T;
   };
   // Each thread copies APT 16-byte pieces of A and CPT - APT of B per slice,
   // all in the same k column, RSTEP rows apart.
-  constexpr int CPT = (TM + TN) * (TK / 2) / NTHREADS;
-  constexpr int APT = TM * (TK / 2) / NTHREADS;
-  constexpr int RSTEP = NTHREADS / (TK / 2);
-  static_assert(CPT * NTHREADS == (TM + TN) * (TK / 2) && APT * NTHREADS == TM * (TK / 2),
+  constexpr int CPT = (TM + TNG) * (TKG / 2) / NTHREADS;
+  constexpr int APT = TM * (TKG / 2) / NTHREADS;
+  constexpr int RSTEP = NTHREADS / (TKG / 2);
+  static_assert(CPT * NTHREADS == (TM + TNG) * (TKG / 2) && APT * NTHREADS == TM * (TKG / 2),
                 "the copies must split evenly over the threads");
-  const int crow0 = tid / (TK / 2), ckc = (tid % (TK / 2)) * 2;
+  const int crow0 = tid / (TKG / 2), ckc = (tid % (TKG / 2)) * 2;
   auto issue = [&](const Tile& T, int slice, int stage) {
-    const int k = slice * TK + ckc;
+    const int k = slice * TKG + ckc;
     const bool kin = k < T.K;
     const uint32_t sa = smem_u32(As + stage * TM * LDS) + (crow0 * LDS + ckc) * 8;
-    const uint32_t sb = smem_u32(Bs + stage * TN * LDS) + (crow0 * LDS + ckc) * 8;
+    const uint32_t sb = smem_u32(Bs + stage * TNG * LDS) + (crow0 * LDS + ckc) * 8;
 #pragma unroll
     for (int i = 0; i < APT; ++i) {
       const int grow = T.m0 + crow0 + i * RSTEP;
@@ -554,20 +584,21 @@ dgemm_nt_kernel(const __grid_constant__ GemmBatch batch) {
   };
   auto prologue = [&](const Tile& T, int g0) {
 #pragma unroll
-    for (int st = 0; st < GSTAGES - 1; ++st) {
-      if (st < T.ns) issue(T, st, (g0 + st) % GSTAGES);
+    for (int st = 0; st < STG - 1; ++st) {
+      if (st < T.ns) issue(T, st, (g0 + st) % STG);
       cp_async_commit();
     }
     if (T.beta != 0.0) {  // pull this tile of C into L2 for the epilogue
-      for (int c = tid; c < TM * 8; c += NTHREADS) {
-        const int row = c >> 3, col = T.n0 + (c & 7) * 16;
+      constexpr int CH = TNG / 16;  // 128-byte pieces per tile row
+      for (int c = tid; c < TM * CH; c += NTHREADS) {
+        const int row = c / CH, col = T.n0 + (c % CH) * 16;
         if (T.m0 + row < T.M && col < T.N)
           asm volatile("prefetch.global.L2 [%0];" ::"l"(T.C + static_cast<long long>(T.m0 + row) * T.ldc + col));
       }
     }
   };
 
-  int g = 0;  // running slice count: stage of a slice = its running index mod GSTAGES
+  int g = 0;  // running slice count: stage of a slice = its running index mod STG
   Tile cur;
   if (t < total) { cur = decode(t); prologue(cur, g); }
   while (t < total) {
@@ -578,13 +609,13 @@ dgemm_nt_kernel(const __grid_constant__ GemmBatch batch) {
 #pragma unroll
       for (int j = 0; j < NI; ++j) acc[i][j][0] = acc[i][j][1] = 0.0;
     for (int sl = 0; sl < cur.ns; ++sl) {
-      cp_async_wait<GSTAGES - 2>();
-      __syncthreads();
-      if (sl + GSTAGES - 1 < cur.ns) issue(cur, sl + GSTAGES - 1, (g + sl + GSTAGES - 1) % GSTAGES);
+      cp_async_wait<STG - 2>();
+      group_sync();
+      if (sl + STG - 1 < cur.ns) issue(cur, sl + STG - 1, (g + sl + STG - 1) % STG);
       cp_async_commit();
-      const int stg = (g + sl) % GSTAGES;
+      const int stg = (g + sl) % STG;
       const double* a_s = As + stg * TM * LDS + (wm * WM + (lane >> 2)) * LDS + (lane & 3);
-      const double* b_s = Bs + stg * TN * LDS + (wn * WN + (lane >> 2)) * LDS + (lane & 3);
+      const double* b_s = Bs + stg * TNG * LDS + (wn * WN + (lane >> 2)) * LDS + (lane & 3);
       // fragments double-buffered: step kk+1's loads are in flight while
       // step kk's MMAs issue
       double af[2][MI], bf[2][NI];
@@ -593,9 +624,9 @@ dgemm_nt_kernel(const __grid_constant__ GemmBatch batch) {
 #pragma unroll
       for (int j = 0; j < NI; ++j) bf[0][j] = b_s[j * 8 * LDS];
 #pragma unroll
-      for (int kk = 0; kk < TK / 4; ++kk) {
+      for (int kk = 0; kk < TKG / 4; ++kk) {
         const int cb = kk & 1;
-        if (kk + 1 < TK / 4) {
+        if (kk + 1 < TKG / 4) {
 #pragma unroll
           for (int i = 0; i < MI; ++i) af[cb ^ 1][i] = a_s[i * 8 * LDS + (kk + 1) * 4];
 #pragma unroll
@@ -608,11 +639,13 @@ dgemm_nt_kernel(const __grid_constant__ GemmBatch batch) {
       }
     }
     g += cur.ns;
-    // start the next tile's copies before this tile's epilogue
+    // one group: start the next tile's copies before this tile's epilogue;
+    // several: after it (the other group's MMAs cover the epilogue, and the
+    // next tile's fields are not held in registers across it)
     const int next = t + step;
-    __syncthreads();  // all warps are done reading the stages
+    group_sync();  // the group's warps are done reading the stages
     Tile nxt;
-    if (next < total) { nxt = decode(next); prologue(nxt, g); }
+    if (NG == 1 && next < total) { nxt = decode(next); prologue(nxt, g); }
 
     // epilogue: lane holds C[8i + lane/4][8j + 2(lane%4) + {0,1}] of its warp
     // block; C is read two row groups at a time so the loads overlap.
@@ -649,6 +682,7 @@ dgemm_nt_kernel(const __grid_constant__ GemmBatch batch) {
         }
       }
     }
+    if (NG > 1 && next < total) { nxt = decode(next); prologue(nxt, g); }
     t = next;
     cur = nxt;
   }

@@ -27,6 +27,14 @@ namespace {
 
 using namespace gptq;
 
+// Shape of the factorization's trailing-update DGEMM (U_k): TM, WGM, warps
+// per group, tile columns, groups, K slice, stages.
+#ifndef GPTQ_UK_SHAPE
+#define GPTQ_UK_SHAPE 128, 4, 8, 64, 2, 16, 3
+#endif
+template <int TM, int WGM, int NW, int TNG, int NG, int TKG, int STG>
+constexpr int gemm_smem_of() { return chol::gemm_smem<TM, TNG, NG, TKG, STG>(); }
+
 constexpr size_t kAlign = 256;
 inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
@@ -104,9 +112,9 @@ gptq_status device_setup(int* num_sms) {
     GPTQ_CUDA_TRY(cudaFuncSetAttribute(syrk::syrk_bf16_tcgen05_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        syrk::SMEM_BYTES));
-    GPTQ_CUDA_TRY(cudaFuncSetAttribute(chol::dgemm_nt_kernel<128, 4, 16>,
+    GPTQ_CUDA_TRY(cudaFuncSetAttribute(chol::dgemm_nt_kernel<GPTQ_UK_SHAPE>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       chol::gemm_smem<128>()));
+                                       gemm_smem_of<GPTQ_UK_SHAPE>()));
     GPTQ_CUDA_TRY(cudaFuncSetAttribute(chol::dgemm_nt_kernel<128, 2>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        chol::gemm_smem<128>()));
@@ -287,7 +295,8 @@ namespace {
 // it (a persistent grid on every SM would keep a later kernel on another
 // stream from starting until it exits).  Problems with an empty output are
 // dropped.
-template <int TM, int WGM, int NW = 8>
+template <int TM, int WGM, int NW = 8, int TNG = chol::TN, int NG = 1, int TKG = chol::TK,
+          int STG = chol::GSTAGES>
 gptq_status launch_nt(const std::vector<chol::GemmProblem>& probs, cudaStream_t s,
                       int reserve_sms = 0) {
   int num_sms = 148;
@@ -300,15 +309,16 @@ gptq_status launch_nt(const std::vector<chol::GemmProblem>& probs, cudaStream_t 
     while (i < probs.size() && b.count < chol::MAXP) {
       const chol::GemmProblem& q = probs[i++];
       if (q.M <= 0 || q.N <= 0) continue;
-      const int tm = (q.M + TM - 1) / TM, tn = (q.N + chol::TN - 1) / chol::TN;
+      const int tm = (q.M + TM - 1) / TM, tn = (q.N + TNG - 1) / TNG;
       b.tile_start[b.count] = tiles;
       b.p[b.count++] = q;
-      tiles += q.lower_only ? tm * (tm + 1) / 2 : tm * tn;
+      tiles += q.lower_only ? chol::lower_tiles<TM, TNG>(q.M, q.N) : tm * tn;
     }
     b.tile_start[b.count] = tiles;
-    const int grid = std::min(tiles, std::max(1, num_sms - reserve_sms));
+    const int grid = std::min((tiles + NG - 1) / NG, std::max(1, num_sms - reserve_sms));
     if (grid > 0) {
-      chol::dgemm_nt_kernel<TM, WGM, NW><<<grid, NW * 32, chol::gemm_smem<TM>(), s>>>(b);
+      chol::dgemm_nt_kernel<TM, WGM, NW, TNG, NG, TKG, STG>
+          <<<grid, NG * NW * 32, chol::gemm_smem<TM, TNG, NG, TKG, STG>(), s>>>(b);
       GPTQ_LAUNCH_CHECK();
     }
   }
@@ -717,7 +727,7 @@ gptq_status gptq_prepare_hinv(const float* H, int64_t d, double damp_rel, float*
     }
     // two SMs stay free for D_k and leaf k+1 on the auxiliary stream (the
     // leaf's 141 KB of shared memory cannot share an SM with a U_k CTA)
-    st = launch_nt<128, 4, 16>(uk, s, 2);
+    st = launch_nt<GPTQ_UK_SHAPE>(uk, s, 2);
     if (st != GPTQ_OK) return st;
     GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, evL[k & 1], 0));  // X_{k+1} for P_{k+1}
   }

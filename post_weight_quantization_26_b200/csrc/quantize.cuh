@@ -9,10 +9,12 @@
 //       lazy-update window, the errors of the whole previous window;
 //   (b) the B columns of every row: parameters at a group start, code,
 //       dequantize, e = (w - w^)/G_qq, subtract e * G[q, k] from the later
-//       columns of the block, keep e in E.  A row's values live in
-//       registers of 4 threads (interleaved in 4-column chunks); G's
+//       columns of the block, keep e in E.  One warp sweeps, one thread per
+//       row, 16 columns at a time in registers, so the dependent chain from
+//       one column to the next crosses no other thread; three warps apply
+//       each finished 16 columns' errors to the rest of the block.  G's
 //       diagonal block sits in shared memory and is read as broadcast
-//       float4s; e crosses the 4 threads by shuffle;
+//       float4s;
 //   (c) write E as a TF32 split for the trailing update and bit-pack the
 //       block's codes.
 // The columns right of block j0 + B are updated by trailing_tf32x3_kernel
@@ -98,17 +100,16 @@ __global__ void prepare_rows_kernel(const float* __restrict__ W, float* __restri
 }
 
 // ------------------------------------------------------------- block step
-// One block of B columns for a slab of QROWS rows (4 threads per row; thread
-// t of a row owns columns 16c + 4t .. 16c + 4t + 3 of the block):
+// One block of B columns for a slab of QROWS rows (4 warps; the staging and
+// the write-out run 4 threads per row, the sweep one thread per row):
 //   (a) if a previous block exists, apply its errors to this block only:
 //       W[rows, blk] -= E_prev[rows] * G[prev blk, blk]  (the columns
 //       further right get them from the trailing-update kernel);
-//   (b) quantize the block column by column in 16-column sub-blocks: per
-//       column the owner codes w_q, e = (w_q - w^_q) / G_qq is broadcast to
-//       the row's 4 threads, each updates its later columns of the
-//       sub-block in registers; after each sub-block one rank-16 update
-//       carries its errors to the rest of the block (same sums as
-//       column-at-a-time, grouped);
+//   (b) quantize the block column by column in 16-column sub-blocks: the
+//       sweeping thread codes w_q, takes e = (w_q - w^_q) / G_qq and updates
+//       the sub-block's later columns in its registers; one rank-16 update
+//       per sub-block (by the helper warps) carries its errors to the rest
+//       of the block (same sums as column-at-a-time, grouped);
 //   (c) bit-pack the block's codes and write E for the trailing update.
 // Group parameters are taken from the current weights when a group's first
 // column is reached (always a sub-block start, as groups are multiples of 32).
@@ -337,99 +338,129 @@ block_step_kernel(const float* __restrict__ Wk, int d_row, int d_col, int j0, in
     __syncthreads();
   }
   for (int q = tid; q < ncols; q += QTHREADS) invd[q] = 1.0f / Gs[q * LDG + q];
-
-  const float maxq = static_cast<float>((1 << bits) - 1);
-  float s = 1.0f, z = 0.0f;
-  if (pc_mode) {
-    if (rv) { s = scales[r]; z = static_cast<float>(zeros[r]); }
-  } else if (group > B && (j0 % group) != 0) {  // the group began in an earlier block
-    const int g = j0 / group;
-    if (rv) { s = scales[static_cast<size_t>(r) * n_groups + g];
-              z = static_cast<float>(zeros[static_cast<size_t>(r) * n_groups + g]); }
-  }
   __syncthreads();
 
-  // (b) 16-column sub-blocks
-  for (int q0 = 0; q0 < ncols; q0 += 16) {
-    if (!pc_mode && ((j0 + q0) % group) == 0) {  // a group starts here
-      const int gend = min(q0 + group, ncols);
-      float mn = 3.4e38f, mx = -3.4e38f;
-      for (int c = q0 + 4 * t; c < gend; c += 16) {
-        const float4 v = *reinterpret_cast<const float4*>(wrow + c);
-        mn = fminf(mn, fminf(fminf(v.x, v.y), fminf(v.z, v.w)));
-        mx = fmaxf(mx, fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
-      }
-      if (group > B && rv) {  // the rest of the group lies right of this block
-        const float* rest = Wk + static_cast<size_t>(r) * d_col;
-        for (int c = j0 + B + t; c < j0 + group; c += 4) {
-          const float v = rest[c];
-          mn = fminf(mn, v); mx = fmaxf(mx, v);
+  // (b) 16-column sub-blocks.  Warp 0 sweeps: lane l holds row r0 + l, takes
+  // a sub-block's 16 values into registers and runs its dependent column
+  // steps with no exchange between threads.  Warps 1..3 apply each finished
+  // sub-block's 16 errors to the block's later columns (a rank-16 update,
+  // lane l again on row r0 + l, 4-column chunks split over the 3 warps).
+  // Two named barriers hand the work over: 1 = "the errors of sub-block sb
+  // are in E", 2 = "the columns of sub-block sb + 1 carry every earlier
+  // error".  The helpers update the next sub-block's columns first and
+  // release the sweeper before the rest, except where a group starts at the
+  // next sub-block: its parameters read the whole group, so they release it
+  // after all their updates.
+  const float maxq = static_cast<float>((1 << bits) - 1);
+  const int warp_id = tid >> 5;
+  const int nsb = ncols / 16;
+  float* hw = Ws + lane * LDG;  // this thread's row in (b)
+  float* he = Es + lane * LDG;
+  if (warp_id == 0) {
+    const int rs = r0 + lane;
+    const bool rvs = rs < d_row;
+    float s = 1.0f, z = 0.0f;
+    if (pc_mode) {
+      if (rvs) { s = scales[rs]; z = static_cast<float>(zeros[rs]); }
+    } else if (group > B && (j0 % group) != 0) {  // the group began in an earlier block
+      const int g = j0 / group;
+      if (rvs) { s = scales[static_cast<size_t>(rs) * n_groups + g];
+                 z = static_cast<float>(zeros[static_cast<size_t>(rs) * n_groups + g]); }
+    }
+    uint32_t* crow = reinterpret_cast<uint32_t*>(codes + lane * L::LDC);
+    for (int sb = 0; sb < nsb; ++sb) {
+      const int q0 = 16 * sb;
+      if (sb > 0) named_bar(2, QTHREADS);
+      if (!pc_mode && ((j0 + q0) % group) == 0) {  // a group starts here
+        const int gend = min(q0 + group, ncols);
+        float mn = 3.4e38f, mx = -3.4e38f;
+        for (int c = q0; c < gend; c += 4) {
+          const float4 v = *reinterpret_cast<const float4*>(hw + c);
+          mn = fminf(mn, fminf(fminf(v.x, v.y), fminf(v.z, v.w)));
+          mx = fmaxf(mx, fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
+        }
+        if (group > B && rvs) {  // the rest of the group lies right of this block
+          const float* rest = Wk + static_cast<size_t>(rs) * d_col;
+          for (int c = j0 + B; c < j0 + group; c += 4) {
+            const float4 v = *reinterpret_cast<const float4*>(rest + c);
+            mn = fminf(mn, fminf(fminf(v.x, v.y), fminf(v.z, v.w)));
+            mx = fmaxf(mx, fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
+          }
+        }
+        make_params(mn, mx, bits, sym, s, z);
+        if (rvs) {
+          const int g = (j0 + q0) / group;
+          scales[static_cast<size_t>(rs) * n_groups + g] = s;
+          zeros[static_cast<size_t>(rs) * n_groups + g] = static_cast<uint8_t>(z);
         }
       }
-      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 2));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      make_params(mn, mx, bits, sym, s, z);
-      if (rv && t == 0) {
-        const int g = (j0 + q0) / group;
-        scales[static_cast<size_t>(r) * n_groups + g] = s;
-        zeros[static_cast<size_t>(r) * n_groups + g] = static_cast<uint8_t>(z);
-      }
-    }
-    float4 wv = *reinterpret_cast<const float4*>(wrow + q0 + 4 * t);
-    float w[4] = {wv.x, wv.y, wv.z, wv.w};
+      float w[16], iv[16], ev[16];
 #pragma unroll
-    for (int u = 0; u < 16; ++u) {
-      const int q = q0 + u;
-      const int tq = u >> 2;
-      // loads first (independent of this column's result), then the
-      // quantization on every lane, branch-free; the owner's result is kept
-      const float4 g4 = *reinterpret_cast<const float4*>(Gs + q * LDG + q0 + 4 * t);
-      const float iq = invd[q];
-      const bool own = (t == tq);
-      const float x = w[u & 3];
-      float qf = rintf(x / s) + z;
-      qf = fminf(fmaxf(qf, 0.0f), maxq);
-      const float xh = s * (qf - z);
-      const float eo = (x - xh) * iq;
-      if (own) {
-        codes[rloc * L::LDC + q] = static_cast<uint8_t>(qf);
-        erow[q] = eo;
+      for (int i = 0; i < 4; ++i) {
+        const float4 v = *reinterpret_cast<const float4*>(hw + q0 + 4 * i);
+        w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+        const float4 d = *reinterpret_cast<const float4*>(invd + q0 + 4 * i);
+        iv[4 * i] = d.x; iv[4 * i + 1] = d.y; iv[4 * i + 2] = d.z; iv[4 * i + 3] = d.w;
       }
-      const float e = __shfl_sync(0xffffffffu, own ? eo : 0.0f, qbase | tq);
-      if (u < 15) {
-        const int kb = 4 * t;
-        w[0] = (kb > u) ? fmaf(-e, g4.x, w[0]) : w[0];
-        w[1] = (kb + 1 > u) ? fmaf(-e, g4.y, w[1]) : w[1];
-        w[2] = (kb + 2 > u) ? fmaf(-e, g4.z, w[2]) : w[2];
-        w[3] = (kb + 3 > u) ? fmaf(-e, g4.w, w[3]) : w[3];
+      uint32_t cw[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const float x = w[u];
+        float qf = rintf(x / s) + z;
+        qf = fminf(fmaxf(qf, 0.0f), maxq);
+        const float xh = s * (qf - z);
+        const float e = (x - xh) * iv[u];
+        ev[u] = e;
+        cw[u >> 2] |= static_cast<uint32_t>(qf) << (8 * (u & 3));
+        // the later columns of the sub-block: w -= e G[q, later]
+        const float* grow = Gs + (q0 + u) * LDG + q0;
+#pragma unroll
+        for (int i = (u + 1) >> 2; i < 4; ++i) {
+          const float4 g4 = *reinterpret_cast<const float4*>(grow + 4 * i);
+          const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            if (4 * i + k > u) w[4 * i + k] = fmaf(-e, gv[k], w[4 * i + k]);
+        }
       }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        *reinterpret_cast<float4*>(he + q0 + 4 * i) =
+            make_float4(ev[4 * i], ev[4 * i + 1], ev[4 * i + 2], ev[4 * i + 3]);
+        crow[q0 / 4 + i] = cw[i];
+      }
+      if (sb + 1 < nsb) named_bar_arrive(1, QTHREADS);
     }
-    __syncwarp();
-    // rank-16 update of the rest of the block: thread t takes chunks
-    // q0/4 + 4 + t, +4, ... (the chunk it owns in the next sub-block first)
-    if (q0 + 16 < ncols) {
+  } else {
+    const int h = warp_id - 1;  // 0..2
+    for (int sb = 0; sb + 1 < nsb; ++sb) {
+      const int q0 = 16 * sb;
+      named_bar(1, QTHREADS);
       float ev[16];
 #pragma unroll
-      for (int u = 0; u < 16; u += 4) {
-        const float4 v = *reinterpret_cast<const float4*>(erow + q0 + u);
-        ev[u] = v.x; ev[u + 1] = v.y; ev[u + 2] = v.z; ev[u + 3] = v.w;
+      for (int i = 0; i < 4; ++i) {
+        const float4 v = *reinterpret_cast<const float4*>(he + q0 + 4 * i);
+        ev[4 * i] = v.x; ev[4 * i + 1] = v.y; ev[4 * i + 2] = v.z; ev[4 * i + 3] = v.w;
       }
-      for (int c = q0 + 16 + 4 * t; c < ncols; c += 16) {
-        float4 acc = *reinterpret_cast<const float4*>(wrow + c);
+      // W[row, c..c+3] -= sum_u e_u G[q0 + u, c..c+3], u in order
+      auto update = [&](int c) {
+        float4 acc = *reinterpret_cast<const float4*>(hw + c);
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
           const float4 g4 = *reinterpret_cast<const float4*>(Gs + (q0 + u) * LDG + c);
           acc.x = fmaf(-ev[u], g4.x, acc.x); acc.y = fmaf(-ev[u], g4.y, acc.y);
           acc.z = fmaf(-ev[u], g4.z, acc.z); acc.w = fmaf(-ev[u], g4.w, acc.w);
         }
-        *reinterpret_cast<float4*>(wrow + c) = acc;
-      }
+        *reinterpret_cast<float4*>(hw + c) = acc;
+      };
+      const bool group_next = !pc_mode && ((j0 + q0 + 16) % group) == 0;
+      for (int ci = h; ci < 4; ci += 3) update(q0 + 16 + 4 * ci);
+      if (!group_next) named_bar_arrive(2, QTHREADS);
+      for (int c = q0 + 32 + 4 * h; c < ncols; c += 12) update(c);
+      if (group_next) named_bar_arrive(2, QTHREADS);
     }
-    __syncwarp();
   }
-
+  __syncthreads();
   // (c) E for the trailing update as a TF32 split (hi = low 13 mantissa bits
   // cleared, lo = E - hi), and the packed codes
   if (rv) {
