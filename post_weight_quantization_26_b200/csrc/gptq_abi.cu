@@ -139,6 +139,17 @@ gptq_status device_setup(int* num_sms) {
     GPTQ_CUDA_TRY(cudaFuncSetAttribute(trail::trailing_tf32x3_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        trail::SMEM_BYTES));
+    // The column sweep runs a step CTA and a trailing-update CTA side by side
+    // on each SM (two streams).  Their shared memory only fits together with
+    // the largest shared-memory carveout; left to itself the driver may size
+    // an SM's carveout for the first kernel alone, and the other then waits
+    // for that SM to drain.
+    for (const void* f : {reinterpret_cast<const void*>(quant::block_step_kernel<128>),
+                          reinterpret_cast<const void*>(quant::block_step_kernel<64>),
+                          reinterpret_cast<const void*>(quant::block_step_kernel<32>),
+                          reinterpret_cast<const void*>(trail::trailing_tf32x3_kernel)})
+      GPTQ_CUDA_TRY(cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                         cudaSharedmemCarveoutMaxShared));
     GPTQ_CUDA_TRY(cudaStreamCreateWithFlags(&di.aux, cudaStreamNonBlocking));
     for (int i = 0; i < kEvents; ++i)
       GPTQ_CUDA_TRY(cudaEventCreateWithFlags(&di.ev[i], cudaEventDisableTiming));
@@ -462,7 +473,7 @@ gptq_status gptq_awq_search(const float* W, const float* H, const double* sx, in
                           CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B)) != GPTQ_OK ||
       (st = encode_f32_2d(&tm_hlo, Hlo, dc, dc, dc, trail::B_BOX, trail::BK,
                           CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B)) != GPTQ_OK ||
-      (st = encode_f32_2d(&tm_t, T, dc, dr, dc, trail::OUT_COLS, trail::BM, CU_TENSOR_MAP_SWIZZLE_128B)) != GPTQ_OK)
+      (st = encode_f32_2d(&tm_t, T, dc, dr, dc, trail::OUT_COLS, trail::OUT_ROWS, CU_TENSOR_MAP_SWIZZLE_128B)) != GPTQ_OK)
     return st;
   trail::Params tp{};
   tp.M = dr; tp.N = dc; tp.K = dc; tp.n0 = 0; tp.j0 = 0;
@@ -792,7 +803,7 @@ gptq_status gptq_quantize_layer(const float* W, int64_t d_row, int64_t d_col, co
                           CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B)) != GPTQ_OK) return st;
   if ((st = encode_f32_2d(&tm_glo, Glo, dc, dc, dc, trail::B_BOX, trail::BK,
                           CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B)) != GPTQ_OK) return st;
-  if ((st = encode_f32_2d(&tm_w, Wk, dc, dr, dc, trail::OUT_COLS, trail::BM,
+  if ((st = encode_f32_2d(&tm_w, Wk, dc, dr, dc, trail::OUT_COLS, trail::OUT_ROWS,
                           CU_TENSOR_MAP_SWIZZLE_128B)) != GPTQ_OK) return st;
   DeviceInfo* di = current_device_info();
   if (!di) return GPTQ_ERR_CUDA;

@@ -19,11 +19,13 @@
 //               used by alternate tiles so that one tile's epilogue overlaps
 //               the next tile's MMAs) and issues tcgen05.mma kind::tf32 from
 //               one thread;
-//   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, negate, write a
-//               128x32 tile to shared memory (128-byte swizzle), and add it
-//               into W with a TMA reduce-add (the L2 does the read-modify-
-//               write).  A long K is summed in chains of `chain` K-steps,
-//               each added into W on its own, in order.
+//   warps 2..5  epilogue, each on its own 32 rows (its TMEM lane quarter):
+//               tcgen05.ld 32 columns at a time, negate, write a 32x32 piece
+//               to its own 4 KB of shared memory (128-byte swizzle), and add
+//               it into W with its own TMA reduce-add (the L2 does the read-
+//               modify-write); no barrier between the four warps.  A long K
+//               is summed in chains of `chain` K-steps, each added into W on
+//               its own, in order.
 // Shared memory is kept near 112 KB so a block-step CTA fits on the same SM
 // (the two kernels run concurrently on different streams).  Every mbarrier
 // wait is bounded.
@@ -42,7 +44,8 @@ constexpr int B_BOX_BYTES = B_BOX * BK * 4;        // 2 KB
 constexpr int B_BYTES = BN * BK * 4;               // 16 KB (one split)
 constexpr int STAGE_BYTES = 2 * A_BYTES + 2 * B_BYTES;  // 48 KB
 constexpr int OUT_COLS = 32;
-constexpr int OUT_BYTES = BM * OUT_COLS * 4;       // 16 KB
+constexpr int OUT_ROWS = 32;                       // rows of one epilogue warp's W box
+constexpr int OUT_BYTES = BM * OUT_COLS * 4;       // 16 KB: 4 warps x 4 KB
 constexpr int NUM_THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + OUT_BYTES + 1024 + 256;
@@ -201,48 +204,53 @@ trailing_tf32x3_kernel(const __grid_constant__ CUtensorMap tm_ehi,
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    const int quarter = warp & 3;  // TMEM lanes [32*quarter, +32) = rows of the tile
-    const int row = quarter * 32 + lane;
-    const bool issuer = (warp == 2 && lane == 0);
-    // The four epilogue warps meet at named barriers, so a warp whose wait
-    // gave up keeps looping (skipping the work) rather than leave the others
-    // waiting at a barrier it will not reach.
+    // Warp q (= warp & 3) owns TMEM lanes [32q, 32q + 32), rows 32q.. of the
+    // tile.  It stages its own 32 x 32 piece in its own 4 KB of the output
+    // buffer and adds it into W with its own TMA reduce-add, so the four
+    // warps never wait for one another.  The next piece's TMEM load is in
+    // flight while the warp waits for its previous reduce to read the buffer.
+    const int quarter = warp & 3;
+    float* obuf = out_ptr + quarter * OUT_ROWS * OUT_COLS;
+    const uint32_t obuf_s = outbuf + quarter * OUT_ROWS * OUT_COLS * 4;
     bool ok = true;
     int lu = 0;
     for (int u = blockIdx.x; u < p.tiles; u += gridDim.x) {
      const int tm = u % p.tiles_m, tn = u / p.tiles_m;
+     const int row0 = tm * BM + quarter * OUT_ROWS;  // this warp's first row of W
      for (int c0 = 0; c0 < nk; c0 += chain, ++lu) {
       const uint32_t acc = lu & 1;
       if (ok && !mbar_wait_bounded(tfull0 + 8u * acc, (lu >> 1) & 1, abort_flag, p.wait_ns)) ok = false;
       tc_fence_after();
-      // a tile's chains land in W in order: the previous chain's adds first
-      if (issuer && c0 > 0) bulk_wait0();
+      // a tile's chains land in W in order: this warp's previous adds first
+      if (lane == 0 && c0 > 0) bulk_wait0();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
       for (int c = 0; c < BN / OUT_COLS; ++c) {
-        if (p.n0 + tn * BN + c * OUT_COLS >= p.n0 + p.N) break;  // past the matrix
+        if (tn * BN + c * OUT_COLS >= p.N) break;  // past the columns to update
         uint32_t r[32];
         if (ok) {
           tmem_ld_32x32b_x32(t_row + c * OUT_COLS, r);
+        }
+        if (lane == 0) bulk_wait_read0();  // the previous reduce has read the buffer
+        __syncwarp();
+        if (ok) {
           tmem_ld_wait();
         } else {
 #pragma unroll
           for (int j = 0; j < 32; ++j) r[j] = 0u;
         }
-        if (issuer) bulk_wait_read0();
-        named_bar(1, 128);  // the previous chunk's reduce has read the buffer
         // 128-byte swizzle: 16-byte chunk j of row r lives at chunk j ^ (r & 7)
-        float* orow = out_ptr + row * OUT_COLS;
+        float* orow = obuf + lane * OUT_COLS;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const int pj = j ^ (row & 7);
+          const int pj = j ^ (lane & 7);
           float4 v = make_float4(-__uint_as_float(r[4 * j]), -__uint_as_float(r[4 * j + 1]),
                                  -__uint_as_float(r[4 * j + 2]), -__uint_as_float(r[4 * j + 3]));
           *reinterpret_cast<float4*>(orow + 4 * pj) = v;
         }
         fence_proxy_async_smem();
-        named_bar(1, 128);
-        if (issuer && ok) {
-          tma_reduce_add_2d(&tm_w, outbuf, p.n0 + tn * BN + c * OUT_COLS, tm * BM);
+        __syncwarp();
+        if (lane == 0 && ok && row0 < p.M) {
+          tma_reduce_add_2d(&tm_w, obuf_s, p.n0 + tn * BN + c * OUT_COLS, row0);
           bulk_commit();
         }
       }
@@ -251,7 +259,7 @@ trailing_tf32x3_kernel(const __grid_constant__ CUtensorMap tm_ehi,
       if (lane == 0) mbar_arrive(tempty0 + 8u * acc);
      }
     }
-    if (issuer) bulk_wait0();
+    if (lane == 0) bulk_wait0();
   }
 
   tc_fence_before();
