@@ -201,7 +201,7 @@ PrepareWs prepare_layout(int64_t d) {
 }
 
 struct QuantWs {
-  size_t Wk, E[2][2], Ghi, Glo, total;  // E[window buffer][hi/lo]
+  size_t Wk, E[2][3], Ghi, Glo, total;  // E[window buffer][hi / lo / as it is]
   int lde;                              // E row stride: one window of blocks
 };
 QuantWs quant_layout(int64_t d_row, int64_t d_col, int block) {
@@ -210,7 +210,7 @@ QuantWs quant_layout(int64_t d_row, int64_t d_col, int block) {
   size_t off = 0;
   w.Wk = off; off = align_up(off + static_cast<size_t>(d_row) * d_col * 4);
   for (int b = 0; b < 2; ++b)
-    for (int h = 0; h < 2; ++h) {
+    for (int h = 0; h < 3; ++h) {
       w.E[b][h] = off;
       off = align_up(off + static_cast<size_t>(d_row) * w.lde * 4);
     }
@@ -277,12 +277,47 @@ gptq_status encode_f32_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint6
   return GPTQ_OK;
 }
 
+// A row-major fp32 matrix (rows x cols, cols a multiple of 32) seen as 3-D
+// for TMA: x = the 32 columns of one 128-byte chunk, y = the row, z = the
+// chunk.  One box of 32 x by x nz lands in shared memory as nz chunks of
+// by rows of 128 bytes, each chunk by * 128 bytes after the previous: the
+// layout of an MN-major operand in 128-byte-swizzled atoms, fetched with one
+// copy instead of nz.
+gptq_status encode_f32_chunks(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows,
+                              uint64_t row_stride, uint32_t by, uint32_t nz,
+                              CUtensorMapSwizzle swz) {
+  const cuuint64_t dims[3] = {32, rows, cols / 32};
+  const cuuint64_t strides[2] = {row_stride * 4, 128};
+  const cuuint32_t box[3] = {32, by, nz};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult cr = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(ptr), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) {
+    std::fprintf(stderr, "gptq: cuTensorMapEncodeTiled (f32 chunks) failed (%d)\n",
+                 static_cast<int>(cr));
+    return GPTQ_ERR_CUDA;
+  }
+  return GPTQ_OK;
+}
+
 // --------------------------------------------------------- SYRK launching
+#ifndef GPTQ_SYRK_CHUNK_CAP
+#define GPTQ_SYRK_CHUNK_CAP 0
+#endif
 void choose_split(int ntiles, int n, int num_sms, int* split_tokens, int* nsplit) {
   const int nkb = (n + syrk::BK - 1) / syrk::BK;
   double best = 1e300;
   int best_s = 1;
   const int max_s = std::max(1, std::min(64, nkb));
+  if (GPTQ_SYRK_CHUNK_CAP > 0 && n > GPTQ_SYRK_CHUNK_CAP) {
+    const int kb_cap = std::max(1, GPTQ_SYRK_CHUNK_CAP / syrk::BK);
+    const int s = (nkb + kb_cap - 1) / kb_cap;
+    const int kb_per = (nkb + s - 1) / s;
+    *split_tokens = kb_per * syrk::BK;
+    *nsplit = (nkb + kb_per - 1) / kb_per;
+    if (static_cast<long long>(ntiles) * *nsplit >= num_sms) return;
+  }
   for (int s = 1; s <= max_s; ++s) {
     const int kb_per = (nkb + s - 1) / s;
     const int s_eff = (nkb + kb_per - 1) / kb_per;
@@ -469,9 +504,9 @@ gptq_status gptq_awq_search(const float* W, const float* H, const double* sx, in
   CUtensorMap tm_ehi, tm_elo, tm_hhi, tm_hlo, tm_t;
   if ((st = encode_f32_2d(&tm_ehi, Ehi, dc, dr, dc, trail::BK, trail::BM, CU_TENSOR_MAP_SWIZZLE_64B)) != GPTQ_OK ||
       (st = encode_f32_2d(&tm_elo, Elo, dc, dr, dc, trail::BK, trail::BM, CU_TENSOR_MAP_SWIZZLE_64B)) != GPTQ_OK ||
-      (st = encode_f32_2d(&tm_hhi, Hhi, dc, dc, dc, trail::B_BOX, trail::BK,
+      (st = encode_f32_chunks(&tm_hhi, Hhi, dc, dc, dc, trail::BK, trail::BN / trail::B_BOX,
                           CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B)) != GPTQ_OK ||
-      (st = encode_f32_2d(&tm_hlo, Hlo, dc, dc, dc, trail::B_BOX, trail::BK,
+      (st = encode_f32_chunks(&tm_hlo, Hlo, dc, dc, dc, trail::BK, trail::BN / trail::B_BOX,
                           CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B)) != GPTQ_OK ||
       (st = encode_f32_2d(&tm_t, T, dc, dr, dc, trail::OUT_COLS, trail::OUT_ROWS, CU_TENSOR_MAP_SWIZZLE_128B)) != GPTQ_OK)
     return st;
@@ -777,9 +812,9 @@ gptq_status gptq_quantize_layer(const float* W, int64_t d_row, int64_t d_col, co
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* base = static_cast<uint8_t*>(ws);
   float* Wk = reinterpret_cast<float*>(base + L.Wk);
-  float* Eb[2][2];
+  float* Eb[2][3];
   for (int b = 0; b < 2; ++b)
-    for (int h = 0; h < 2; ++h) Eb[b][h] = reinterpret_cast<float*>(base + L.E[b][h]);
+    for (int h = 0; h < 3; ++h) Eb[b][h] = reinterpret_cast<float*>(base + L.E[b][h]);
   float* Ghi = reinterpret_cast<float*>(base + L.Ghi);
   float* Glo = reinterpret_cast<float*>(base + L.Glo);
   const int dr = static_cast<int>(d_row), dc = static_cast<int>(d_col);
@@ -799,9 +834,9 @@ gptq_status gptq_quantize_layer(const float* W, int64_t d_row, int64_t d_col, co
                          CU_TENSOR_MAP_SWIZZLE_64B);
       if (st != GPTQ_OK) return st;
     }
-  if ((st = encode_f32_2d(&tm_ghi, Ghi, dc, dc, dc, trail::B_BOX, trail::BK,
+  if ((st = encode_f32_chunks(&tm_ghi, Ghi, dc, dc, dc, trail::BK, trail::BN / trail::B_BOX,
                           CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B)) != GPTQ_OK) return st;
-  if ((st = encode_f32_2d(&tm_glo, Glo, dc, dc, dc, trail::B_BOX, trail::BK,
+  if ((st = encode_f32_chunks(&tm_glo, Glo, dc, dc, dc, trail::BK, trail::BN / trail::B_BOX,
                           CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B)) != GPTQ_OK) return st;
   if ((st = encode_f32_2d(&tm_w, Wk, dc, dr, dc, trail::OUT_COLS, trail::OUT_ROWS,
                           CU_TENSOR_MAP_SWIZZLE_128B)) != GPTQ_OK) return st;
@@ -832,6 +867,7 @@ gptq_status gptq_quantize_layer(const float* W, int64_t d_row, int64_t d_col, co
   const dim3 qgrid((dr + quant::QROWS - 1) / quant::QROWS);
   // W[:, n0:n1] -= E[buf][:, ek0:ek0+K] * G[gj0:gj0+K, n0:n1]
   auto trailing = [&](int buf, int ek0, int K, int gj0, int n0, int n1) -> gptq_status {
+    if (n0 % trail::B_BOX != 0) return GPTQ_ERR_INVALID;  // G is fetched in 32-column chunks
     trail::Params tp{};
     tp.M = dr; tp.N = n1 - n0; tp.K = K; tp.n0 = n0; tp.j0 = gj0; tp.ek0 = ek0;
     tp.chain = 256 / trail::BK;  // a window's update is summed 256 columns at a time
@@ -854,20 +890,21 @@ gptq_status gptq_quantize_layer(const float* W, int64_t d_row, int64_t d_col, co
     if (g > B && j0 % g == 0 && jb >= 1)  // group params read columns ahead
       GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, evT[(jb - 1) % 4], 0));
     // the previous block, or at a window's first block the whole previous window
-    const float *Eph = nullptr, *Epl = nullptr;
+    const float* Ep = nullptr;
     int jp0 = -1, nprev = 0;
     if (jb > 0 && pos > 0) {
-      Eph = Eb[cb][0] + (pos - 1) * B; Epl = Eb[cb][1] + (pos - 1) * B;
+      Ep = Eb[cb][2] + (pos - 1) * B;
       jp0 = j0 - B; nprev = B;
     } else if (jb > 0) {
-      Eph = Eb[pb][0]; Epl = Eb[pb][1];
+      Ep = Eb[pb][2];
       jp0 = e0 - mw * B; nprev = mw * B;
     }
+    float* Ecf = Eb[cb][2] + pos * B;
     float* Ech = Eb[cb][0] + pos * B;
     float* Ecl = Eb[cb][1] + pos * B;
 #define GPTQ_STEP(BB)                                                                        \
   quant::block_step_kernel<BB><<<qgrid, quant::QTHREADS, quant::block_step_smem<BB>(), s>>>( \
-      Wk, dr, dc, j0, ncols, G, Eph, Epl, jp0, nprev, lde, Ech, Ecl, qweight, scales, zeros,  \
+      Wk, dr, dc, j0, ncols, G, Ep, jp0, nprev, lde, Ecf, Ech, Ecl, qweight, scales, zeros,     \
       cfg->bits, cfg->sym, g, n_groups, per_channel)
     if (B == 128) GPTQ_STEP(128);
     else if (B == 64) GPTQ_STEP(64);

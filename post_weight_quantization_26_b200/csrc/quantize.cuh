@@ -110,7 +110,8 @@ __global__ void prepare_rows_kernel(const float* __restrict__ W, float* __restri
 //       the sub-block's later columns in its registers; one rank-16 update
 //       per sub-block (by the helper warps) carries its errors to the rest
 //       of the block (same sums as column-at-a-time, grouped);
-//   (c) bit-pack the block's codes and write E for the trailing update.
+//   (c) bit-pack the block's codes and write E: as it is (for the next
+//       block's step) and as a TF32 split (for the trailing update).
 // Group parameters are taken from the current weights when a group's first
 // column is reached (always a sub-block start, as groups are multiples of 32).
 constexpr int QROWS = 32;            // rows per CTA
@@ -194,9 +195,9 @@ __device__ __forceinline__ void stage_gblock(float* dst, const float* G, int d_c
 template <int B>
 __global__ void __launch_bounds__(QTHREADS)
 block_step_kernel(const float* __restrict__ Wk, int d_row, int d_col, int j0, int ncols,
-                  const float* __restrict__ G, const float* __restrict__ Eprev_hi,
-                  const float* __restrict__ Eprev_lo, int jp0, int nprev, int lde,
-                  float* __restrict__ Ecur_hi, float* __restrict__ Ecur_lo,
+                  const float* __restrict__ G, const float* __restrict__ Eprev, int jp0,
+                  int nprev, int lde, float* __restrict__ Ecur, float* __restrict__ Ecur_hi,
+                  float* __restrict__ Ecur_lo,
                   uint32_t* __restrict__ qweight, float* __restrict__ scales,
                   uint8_t* __restrict__ zeros, int bits, int sym, int group, int n_groups,
                   int pc_mode) {
@@ -211,7 +212,7 @@ block_step_kernel(const float* __restrict__ Wk, int d_row, int d_col, int j0, in
 
   const int tid = threadIdx.x;
   const int rloc = tid >> 2, t = tid & 3;
-  const int lane = tid & 31, qbase = lane & ~3;
+  const int lane = tid & 31;
   const int r0 = blockIdx.x * QROWS;
   const int r = r0 + rloc;
   const bool rv = r < d_row;
@@ -219,7 +220,7 @@ block_step_kernel(const float* __restrict__ Wk, int d_row, int d_col, int j0, in
   // E_prev (nprev columns, row stride lde) and the G rows [jp0, jp0 + nprev)
   // are taken in chunks of B columns
   auto stage_chunk = [&](int kc) {
-    stage_rows<B>(Es, Eprev_hi + kc, lde, r0, d_row, B, tid);
+    stage_rows<B>(Es, Eprev + kc, lde, r0, d_row, B, tid);
     stage_gblock<B>(Gs, G, d_col, jp0 + kc, j0, B, ncols, tid);
   };
   stage_rows<B>(Ws, Wk + j0, d_col, r0, d_row, ncols, tid);
@@ -229,7 +230,6 @@ block_step_kernel(const float* __restrict__ Wk, int d_row, int d_col, int j0, in
   asm volatile("cp.async.wait_group 0;" ::: "memory");
   __syncthreads();
 
-  float* wrow = Ws + rloc * LDG;
   float* erow = Es + rloc * LDG;
   if (nprev > 0) {
     // (a) W[rows, blk] -= E_prev[rows] * G[prev cols, blk] on the MMA path:
@@ -273,19 +273,6 @@ block_step_kernel(const float* __restrict__ Wk, int d_row, int d_col, int j0, in
         for (int nt = 0; nt < NTW; ++nt)
 #pragma unroll
           for (int e = 0; e < 4; ++e) part[mt][nt][e] = 0.0f;
-      // E = E_hi + E_lo (exact): add the low parts in place
-      for (int c = tid; c < QROWS * (B / 4); c += QTHREADS) {
-        const int rr = c / (B / 4), k = (c - rr * (B / 4)) * 4;
-        if (r0 + rr < d_row) {
-          const float4 lo = *reinterpret_cast<const float4*>(
-              Eprev_lo + static_cast<size_t>(r0 + rr) * lde + kc + k);
-          float4* hp = reinterpret_cast<float4*>(Es + rr * L::LDG + k);
-          float4 h = *hp;
-          h.x += lo.x; h.y += lo.y; h.z += lo.z; h.w += lo.w;
-          *hp = h;
-        }
-      }
-      __syncthreads();
       if (cw < ncols) {
 #pragma unroll 2
         for (int k0 = 0; k0 < B; k0 += 8) {
@@ -372,22 +359,26 @@ block_step_kernel(const float* __restrict__ Wk, int d_row, int d_col, int j0, in
       const int q0 = 16 * sb;
       if (sb > 0) named_bar(2, QTHREADS);
       if (!pc_mode && ((j0 + q0) % group) == 0) {  // a group starts here
+        // four independent min/max chains, 16 columns per step (a group
+        // and the block are multiples of 16 columns)
         const int gend = min(q0 + group, ncols);
-        float mn = 3.4e38f, mx = -3.4e38f;
-        for (int c = q0; c < gend; c += 4) {
-          const float4 v = *reinterpret_cast<const float4*>(hw + c);
-          mn = fminf(mn, fminf(fminf(v.x, v.y), fminf(v.z, v.w)));
-          mx = fmaxf(mx, fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
-        }
+        float mn[4] = {3.4e38f, 3.4e38f, 3.4e38f, 3.4e38f};
+        float mx[4] = {-3.4e38f, -3.4e38f, -3.4e38f, -3.4e38f};
+        auto scan16 = [&](const float* p) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float4 v = *reinterpret_cast<const float4*>(p + 4 * i);
+            mn[i] = fminf(mn[i], fminf(fminf(v.x, v.y), fminf(v.z, v.w)));
+            mx[i] = fmaxf(mx[i], fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
+          }
+        };
+        for (int c = q0; c < gend; c += 16) scan16(hw + c);
         if (group > B && rvs) {  // the rest of the group lies right of this block
           const float* rest = Wk + static_cast<size_t>(rs) * d_col;
-          for (int c = j0 + B; c < j0 + group; c += 4) {
-            const float4 v = *reinterpret_cast<const float4*>(rest + c);
-            mn = fminf(mn, fminf(fminf(v.x, v.y), fminf(v.z, v.w)));
-            mx = fmaxf(mx, fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
-          }
+          for (int c = j0 + B; c < j0 + group; c += 16) scan16(rest + c);
         }
-        make_params(mn, mx, bits, sym, s, z);
+        make_params(fminf(fminf(mn[0], mn[1]), fminf(mn[2], mn[3])),
+                    fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), bits, sym, s, z);
         if (rvs) {
           const int g = (j0 + q0) / group;
           scales[static_cast<size_t>(rs) * n_groups + g] = s;
@@ -453,8 +444,25 @@ block_step_kernel(const float* __restrict__ Wk, int d_row, int d_col, int j0, in
         }
         *reinterpret_cast<float4*>(hw + c) = acc;
       };
+      // two chunks with their FMA chains interleaved
+      auto update2 = [&](int c, int c2) {
+        float4 a = *reinterpret_cast<const float4*>(hw + c);
+        float4 b = *reinterpret_cast<const float4*>(hw + c2);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const float4 g4 = *reinterpret_cast<const float4*>(Gs + (q0 + u) * LDG + c);
+          const float4 g5 = *reinterpret_cast<const float4*>(Gs + (q0 + u) * LDG + c2);
+          a.x = fmaf(-ev[u], g4.x, a.x); a.y = fmaf(-ev[u], g4.y, a.y);
+          a.z = fmaf(-ev[u], g4.z, a.z); a.w = fmaf(-ev[u], g4.w, a.w);
+          b.x = fmaf(-ev[u], g5.x, b.x); b.y = fmaf(-ev[u], g5.y, b.y);
+          b.z = fmaf(-ev[u], g5.z, b.z); b.w = fmaf(-ev[u], g5.w, b.w);
+        }
+        *reinterpret_cast<float4*>(hw + c) = a;
+        *reinterpret_cast<float4*>(hw + c2) = b;
+      };
       const bool group_next = !pc_mode && ((j0 + q0 + 16) % group) == 0;
-      for (int ci = h; ci < 4; ci += 3) update(q0 + 16 + 4 * ci);
+      if (h == 0) update2(q0 + 16, q0 + 28);
+      else update(q0 + 16 + 4 * h);
       if (!group_next) named_bar_arrive(2, QTHREADS);
       for (int c = q0 + 32 + 4 * h; c < ncols; c += 12) update(c);
       if (group_next) named_bar_arrive(2, QTHREADS);
@@ -464,11 +472,13 @@ block_step_kernel(const float* __restrict__ Wk, int d_row, int d_col, int j0, in
   // (c) E for the trailing update as a TF32 split (hi = low 13 mantissa bits
   // cleared, lo = E - hi), and the packed codes
   if (rv) {
+    float* ef = Ecur + static_cast<size_t>(r) * lde;
     float* eh = Ecur_hi + static_cast<size_t>(r) * lde;
     float* el = Ecur_lo + static_cast<size_t>(r) * lde;
     for (int c = 4 * t; c < B; c += 16) {
       const float4 v = (c < ncols) ? *reinterpret_cast<const float4*>(erow + c)
                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+      *reinterpret_cast<float4*>(ef + c) = v;
       const float4 h = make_float4(__uint_as_float(__float_as_uint(v.x) & 0xFFFFE000u),
                                    __uint_as_float(__float_as_uint(v.y) & 0xFFFFE000u),
                                    __uint_as_float(__float_as_uint(v.z) & 0xFFFFE000u),

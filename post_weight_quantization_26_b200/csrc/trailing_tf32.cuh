@@ -14,7 +14,9 @@
 //   warp 0      TMA producer: per 16-wide K slice, E_hi/E_lo boxes (K-major,
 //               64-byte swizzle) and G_hi/G_lo boxes (MN-major, 128-byte
 //               swizzle with 32-byte atoms, the one MN-major form tf32
-//               operands take), two-deep ring;
+//               operands take; G is addressed as 32-column chunks x rows x
+//               chunks, so each split's 256 columns come in one copy),
+//               two-deep ring: four copies per K slice;
 //   warp 1      allocates 512 TMEM columns (two fp32 128x256 accumulators,
 //               used by alternate tiles so that one tile's epilogue overlaps
 //               the next tile's MMAs) and issues tcgen05.mma kind::tf32 from
@@ -149,12 +151,10 @@ trailing_tf32x3_kernel(const __grid_constant__ CUtensorMap tm_ehi,
           const uint32_t s0 = ring + stage * STAGE_BYTES;
           tma_load_2d(s0, &tm_ehi, fb, p.ek0 + ks * BK, tm * BM);
           tma_load_2d(s0 + A_BYTES, &tm_elo, fb, p.ek0 + ks * BK, tm * BM);
-          const int gx = p.n0 + tn * BN, gy = p.j0 + ks * BK;
-#pragma unroll
-          for (int c = 0; c < BN / B_BOX; ++c) {
-            tma_load_2d(s0 + 2 * A_BYTES + c * B_BOX_BYTES, &tm_ghi, fb, gx + c * B_BOX, gy);
-            tma_load_2d(s0 + 2 * A_BYTES + B_BYTES + c * B_BOX_BYTES, &tm_glo, fb, gx + c * B_BOX, gy);
-          }
+          // G: all BN / 32 column chunks of the K slice in one copy per split
+          const int gz = (p.n0 + tn * BN) / B_BOX, gy = p.j0 + ks * BK;
+          tma_load_3d(s0 + 2 * A_BYTES, &tm_ghi, fb, 0, gy, gz);
+          tma_load_3d(s0 + 2 * A_BYTES + B_BYTES, &tm_glo, fb, 0, gy, gz);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
