@@ -302,22 +302,11 @@ gptq_status encode_f32_chunks(CUtensorMap* m, const void* ptr, uint64_t cols, ui
 }
 
 // --------------------------------------------------------- SYRK launching
-#ifndef GPTQ_SYRK_CHUNK_CAP
-#define GPTQ_SYRK_CHUNK_CAP 0
-#endif
 void choose_split(int ntiles, int n, int num_sms, int* split_tokens, int* nsplit) {
   const int nkb = (n + syrk::BK - 1) / syrk::BK;
   double best = 1e300;
   int best_s = 1;
   const int max_s = std::max(1, std::min(64, nkb));
-  if (GPTQ_SYRK_CHUNK_CAP > 0 && n > GPTQ_SYRK_CHUNK_CAP) {
-    const int kb_cap = std::max(1, GPTQ_SYRK_CHUNK_CAP / syrk::BK);
-    const int s = (nkb + kb_cap - 1) / kb_cap;
-    const int kb_per = (nkb + s - 1) / s;
-    *split_tokens = kb_per * syrk::BK;
-    *nsplit = (nkb + kb_per - 1) / kb_per;
-    if (static_cast<long long>(ntiles) * *nsplit >= num_sms) return;
-  }
   for (int s = 1; s <= max_s; ++s) {
     const int kb_per = (nkb + s - 1) / s;
     const int s_eff = (nkb + kb_per - 1) / kb_per;
