@@ -768,7 +768,9 @@ def run_w4a16(args, rank, world, local_rank):
                    "batch": batch, "l2": "inputs larger than L2 (271 MB of packed layers per step)",
                    "parallelism": f"{world} independent replica(s), one per GPU"},
         "per_layer_us": dict(zip([n for n, _, _ in W4_LAYERS], per_layer_us)),
-        "roofline": {"bound": "hbm", "kernel": f"w4a16_matmul_kernel ({W4_LAYERS[big][0]})",
+        "roofline": {"bound": "hbm",
+                     "kernel": ("w4a16_wide_kernel" if group == 0 or group % 128 == 0
+                                else "w4a16_matmul_kernel") + f" ({W4_LAYERS[big][0]})",
                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": kernel_traffic(f"w4a16_matmul_kernel/{W4_LAYERS[big][0]}",
                                                "post_weight_quantization_26_b200/csrc/w4a16.cuh"),

@@ -406,6 +406,18 @@ gptq_status gptq_w4a16_matmul(const uint32_t* qweight, const float* scales,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int dr = static_cast<int>(d_row), dc = static_cast<int>(d_col), nb = static_cast<int>(batch);
   const int g = cfg->group_size, n_groups = g ? dc / g : 1;
+  if (g == 0 || g % 128 == 0) {
+    // scale regions of whole 128-column chunks: the unstaged layout
+    const int grid = (dr + w4a16::W_ROWS - 1) / w4a16::W_ROWS;
+    if (g == 0)
+      w4a16::w4a16_wide_kernel<true><<<grid, w4a16::THREADS, 0, s>>>(
+          qweight, scales, zeros, static_cast<const __nv_bfloat16*>(X), Y, dr, dc, nb, g, n_groups);
+    else
+      w4a16::w4a16_wide_kernel<false><<<grid, w4a16::THREADS, 0, s>>>(
+          qweight, scales, zeros, static_cast<const __nv_bfloat16*>(X), Y, dr, dc, nb, g, n_groups);
+    GPTQ_LAUNCH_CHECK();
+    return GPTQ_OK;
+  }
   const int tiles = (dr + w4a16::ROWS - 1) / w4a16::ROWS;
   // two 128-column chunks per work item where the scale regions are whole
   // chunks and the activations leave room for a deep ring; one otherwise

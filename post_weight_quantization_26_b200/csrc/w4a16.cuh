@@ -398,5 +398,179 @@ w4a16_matmul_kernel(const uint32_t* __restrict__ qweight, const float* __restric
   cp_async_wait(0);
 }
 
+// ------------------------------------------------------------------------
+// Layers with one scale per output channel, or per group of a multiple of
+// 128 columns (the common GPTQ settings): a leaner layout with no staging.
+//
+// A CTA owns 32 rows (two 16-row mma tiles per warp) and its 8 warps split
+// the 128-column chunks of the row (warp w: chunks w, w + 8, ...); one
+// shared-memory sum over the warps at the end gives Y.  Lane (g, t) loads,
+// for rows g and g + 8 of each tile, the 16 bytes holding words 4t..4t+3 of
+// the chunk (columns 32t..32t+31): a quad reads 64 contiguous bytes of a row
+// with one 128-bit load each, straight into registers, and the next chunk's
+// loads are issued before the current chunk is computed.  Within a chunk the
+// k order is free (A and B agree on it): mma pair j takes word 4t + j of
+// every lane, slots (2t, 2t+1, 2t+8, 2t+9) holding codes (0, 4, 1, 5) of the
+// word and then (2, 6, 3, 7), so a pair spans the whole chunk, which is why
+// a scale region must cover whole chunks here.  The activations of those
+// columns (batch row g) are loaded and permuted once per chunk and serve
+// both tiles.  Decoding a word: code c of the word becomes the bf16 128 + c
+// with one LOP3 per pair of codes (three shifts per word), and one bf16x2
+// subtraction of 128 + z gives c - z exactly.
+constexpr int WT = 2;             // 16-row tiles per warp
+constexpr int W_ROWS = ROWS * WT;  // rows per CTA
+
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t word_at(const uint4& v, int j) {
+  return j == 0 ? v.x : j == 1 ? v.y : j == 2 ? v.z : v.w;
+}
+
+// Rows g, g + 8 of one tile, word j of the lane's piece: two mma steps.
+__device__ __forceinline__ void tile_word_mma(float (&d)[4], uint32_t vg, uint32_t vh,
+                                              uint32_t zg, uint32_t zh, const uint32_t (&b)[4]) {
+  const uint32_t g0 = bf16x2_sub(code_pair(vg), zg), h0 = bf16x2_sub(code_pair(vh), zh);
+  const uint32_t g1 = bf16x2_sub(code_pair(vg >> 4), zg), h1 = bf16x2_sub(code_pair(vh >> 4), zh);
+  mma_bf16_16816(d, g0, h0, g1, h1, b[0], b[1]);
+  const uint32_t g2 = bf16x2_sub(code_pair(vg >> 8), zg), h2 = bf16x2_sub(code_pair(vh >> 8), zh);
+  const uint32_t g3 = bf16x2_sub(code_pair(vg >> 12), zg), h3 = bf16x2_sub(code_pair(vh >> 12), zh);
+  mma_bf16_16816(d, g2, h2, g3, h3, b[2], b[3]);
+}
+
+template <bool PER_CHANNEL>
+__global__ void __launch_bounds__(THREADS, 2)
+w4a16_wide_kernel(const uint32_t* __restrict__ qweight, const float* __restrict__ scales,
+                  const uint8_t* __restrict__ zeros, const __nv_bfloat16* __restrict__ X,
+                  float* __restrict__ Y, int d_row, int d_col, int batch, int group,
+                  int n_groups) {
+  __shared__ float red[WARPS][WT][32][4];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int words = d_col >> 3;
+  const int nchunks = (d_col + 127) >> 7;
+  const int row0 = blockIdx.x * W_ROWS;
+  // the lane's rows, clamped into the layer for the loads (rows past d_row
+  // are computed on a real row and never written)
+  const uint4* wrow[WT][2];
+  int prow[WT][2];
+#pragma unroll
+  for (int i = 0; i < WT; ++i)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int r = min(row0 + ROWS * i + g + 8 * h, d_row - 1);
+      prow[i][h] = r;
+      wrow[i][h] = reinterpret_cast<const uint4*>(qweight + static_cast<size_t>(r) * words) + t;
+    }
+  const bool xrow_ok = g < batch;
+  const uint4* xrow = reinterpret_cast<const uint4*>(X + static_cast<size_t>(xrow_ok ? g : 0) * d_col) + 4 * t;
+
+  // one chunk's inputs: the lane's weight pieces, its activations, and (for
+  // groups) the scales and zero points of its rows
+  struct In {
+    uint4 w[WT][2];
+    uint4 x[4];
+    float s[WT][2];
+    uint32_t z[WT][2];
+  };
+  auto load = [&](int cc, In& in) {
+    const bool lv = 128 * cc + 32 * t < d_col;  // this lane's 32 columns exist
+#pragma unroll
+    for (int i = 0; i < WT; ++i)
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        in.w[i][h] = lv ? ld_stream_v4(wrow[i][h] + 4 * cc) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      in.x[j] = (lv && xrow_ok) ? __ldg(xrow + 16 * cc + j) : make_uint4(0u, 0u, 0u, 0u);
+    if (!PER_CHANNEL) {
+      const int gi = (128 * cc) / group;
+#pragma unroll
+      for (int i = 0; i < WT; ++i)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const size_t o = static_cast<size_t>(prow[i][h]) * n_groups + gi;
+          in.s[i][h] = __ldg(scales + o);
+          in.z[i][h] = zero_pair(__ldg(zeros + o));
+        }
+    }
+  };
+
+  uint32_t zc[WT][2];
+  if (PER_CHANNEL) {
+#pragma unroll
+    for (int i = 0; i < WT; ++i)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) zc[i][h] = zero_pair(__ldg(zeros + prow[i][h]));
+  }
+  float acc[WT][4];
+#pragma unroll
+  for (int i = 0; i < WT; ++i)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[i][e] = 0.0f;
+
+  In cur, nxt;
+  if (warp < nchunks) load(warp, cur);
+  for (int c = warp; c < nchunks; c += WARPS) {
+    if (c + WARPS < nchunks) load(c + WARPS, nxt);  // in flight while this chunk computes
+    // B fragments of the chunk's 4 words: (x0, x4), (x1, x5), (x2, x6), (x3, x7)
+    uint32_t b[4][4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      b[j][0] = __byte_perm(cur.x[j].x, cur.x[j].z, 0x5410);
+      b[j][1] = __byte_perm(cur.x[j].x, cur.x[j].z, 0x7632);
+      b[j][2] = __byte_perm(cur.x[j].y, cur.x[j].w, 0x5410);
+      b[j][3] = __byte_perm(cur.x[j].y, cur.x[j].w, 0x7632);
+    }
+#pragma unroll
+    for (int i = 0; i < WT; ++i) {
+      if (PER_CHANNEL) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          tile_word_mma(acc[i], word_at(cur.w[i][0], j), word_at(cur.w[i][1], j), zc[i][0],
+                        zc[i][1], b[j]);
+      } else {
+        float part[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          tile_word_mma(part, word_at(cur.w[i][0], j), word_at(cur.w[i][1], j), cur.z[i][0],
+                        cur.z[i][1], b[j]);
+        acc[i][0] = fmaf(cur.s[i][0], part[0], acc[i][0]);
+        acc[i][1] = fmaf(cur.s[i][0], part[1], acc[i][1]);
+        acc[i][2] = fmaf(cur.s[i][1], part[2], acc[i][2]);
+        acc[i][3] = fmaf(cur.s[i][1], part[3], acc[i][3]);
+      }
+    }
+    cur = nxt;
+  }
+  if (PER_CHANNEL) {
+#pragma unroll
+    for (int i = 0; i < WT; ++i) {
+      const float sg = __ldg(scales + prow[i][0]), sh = __ldg(scales + prow[i][1]);
+      acc[i][0] *= sg; acc[i][1] *= sg; acc[i][2] *= sh; acc[i][3] *= sh;
+    }
+  }
+  // sum over the warps.  Fragment element e of lane l is row (l >> 2) +
+  // 8 (e >> 1) of the tile, activation row 2 (l & 3) + (e & 1).
+#pragma unroll
+  for (int i = 0; i < WT; ++i)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) red[warp][i][lane][e] = acc[i][e];
+  __syncthreads();
+  {
+    const int i = threadIdx.x >> 7, l = (threadIdx.x >> 2) & 31, e = threadIdx.x & 3;
+    float y = 0.0f;
+#pragma unroll
+    for (int w = 0; w < WARPS; ++w) y += red[w][i][l][e];
+    const int r = row0 + ROWS * i + (l >> 2) + 8 * (e >> 1), n = 2 * (l & 3) + (e & 1);
+    if (r < d_row && n < batch) Y[static_cast<size_t>(n) * d_row + r] = y;
+  }
+}
+
 }  // namespace w4a16
 }  // namespace gptq
