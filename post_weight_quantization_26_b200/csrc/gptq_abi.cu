@@ -115,9 +115,6 @@ gptq_status device_setup(int* num_sms) {
     GPTQ_CUDA_TRY(cudaFuncSetAttribute(chol::dgemm_nt_kernel<GPTQ_UK_SHAPE>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        gemm_smem_of<GPTQ_UK_SHAPE>()));
-    GPTQ_CUDA_TRY(cudaFuncSetAttribute(chol::dgemm_nt_kernel<128, 2>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       chol::gemm_smem<128>()));
     GPTQ_CUDA_TRY(cudaFuncSetAttribute(chol::dgemm_nt_kernel<64, 2>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        chol::gemm_smem<64>()));
@@ -715,9 +712,11 @@ gptq_status gptq_prepare_hinv(const float* H, int64_t d, double damp_rel, float*
       q.M = k0; q.N = nk; q.K = nk; q.alpha = 1.0; q.beta = 0.0;
       pk.push_back(q);
     }
+    // 64-row tiles from about one wave of them up: the panel is K = 128
+    // deep, so finer tiles balance the SMs better than 128-row ones (at
+    // d = 22016, 342 tiles against 171 on 148 SMs)
     const int prow = rest + k0;
-    if (prow >= 148 * 128) st = launch_nt<128, 2>(pk, s);
-    else if (prow >= 148 * 64) st = launch_nt<64, 2>(pk, s);
+    if (prow >= 148 * 64) st = launch_nt<64, 2>(pk, s);
     else st = launch_nt<32, 1>(pk, s);
     if (st != GPTQ_OK) return st;
     if (rest <= 0) break;
