@@ -84,14 +84,16 @@ diag_stats_kernel(const float* __restrict__ H, int d, double damp_rel,
 __global__ void reverse_damp_fill_kernel(const float* __restrict__ H, int d,
                                          const double* __restrict__ stats,
                                          double* __restrict__ A) {
-  const int i = blockIdx.y;
   const double lam = stats[0];
-  const float* hrow = H + static_cast<size_t>(d - 1 - i) * d;
-  double* arow = A + static_cast<size_t>(i) * d;
-  for (int j = blockIdx.x * blockDim.x + threadIdx.x; j <= i; j += gridDim.x * blockDim.x) {
-    double v = static_cast<double>(hrow[d - 1 - j]);
-    if (j == i) v = (v == 0.0) ? 1.0 : v + lam;
-    arow[j] = v;
+  // rows grid-strided: gridDim.y is capped at 65535 and d may be 65536
+  for (int i = blockIdx.y; i < d; i += gridDim.y) {
+    const float* hrow = H + static_cast<size_t>(d - 1 - i) * d;
+    double* arow = A + static_cast<size_t>(i) * d;
+    for (int j = blockIdx.x * blockDim.x + threadIdx.x; j <= i; j += gridDim.x * blockDim.x) {
+      double v = static_cast<double>(hrow[d - 1 - j]);
+      if (j == i) v = (v == 0.0) ? 1.0 : v + lam;
+      arow[j] = v;
+    }
   }
 }
 

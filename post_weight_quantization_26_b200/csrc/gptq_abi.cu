@@ -671,7 +671,7 @@ gptq_status gptq_prepare_hinv(const float* H, int64_t d, double damp_rel, float*
   chol::diag_stats_kernel<<<1, 1024, 0, s>>>(H, di, damp_rel, dead_mask, stats, istat);
   GPTQ_LAUNCH_CHECK();
   {
-    dim3 grid((di + 255) / 256, di);
+    dim3 grid((di + 255) / 256, std::min(di, 65535));
     chol::reverse_damp_fill_kernel<<<grid, 256, 0, s>>>(H, di, stats, A);
     GPTQ_LAUNCH_CHECK();
   }
