@@ -87,6 +87,12 @@ def parse_args(argv=None):
     p.add_argument("--awq", action="store_true",
                    help="time the AWQ scale search (20-point alpha grid) on the q_proj layer "
                         "with 32768 calibration tokens, 4-bit g128")
+    p.add_argument("--route", choices=["inverse", "factor"], default="factor",
+                   help="factor (default): F, G's diagonal blocks and V_ab G_bb "
+                        "(prepare_factor + quantize_layer_factor), half the fp64 work; "
+                        "inverse: G = chol(H^-1) (prepare_hinv + quantize_layer)")
+    p.add_argument("--no-other-route", action="store_true",
+                   help="skip timing the inverse route beside the factor route")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args(argv)
@@ -127,17 +133,23 @@ def workload_spec(name: str, rank: int):
     return workload_layers(name, rank)[0][0]
 
 
-def work_model(groups):
+def work_model(groups, route="inverse"):
     """Algorithmic work of one step (per stage), counted as the method needs
-    it: the SYRK d(d+1)n flops per input, the factorization 2/3 d^3 fp64 flops
-    per input, the column sweep d_row d_col (d_col - 1) fp32 flops per layer,
-    and the packed output d_row d_col (1 + b/8) bytes per layer."""
+    it: the SYRK d(d+1)n flops per input; the factorization 2/3 d^3 fp64
+    flops per input on the inverse route (Cholesky d^3/3, triangular inverse
+    d^3/3), d^3/3 + 128 d^2 on the factor route (Cholesky, and the panels
+    V_ab G_bb of F: 2 * 128^2 flops per element row of each panel); the
+    column sweep d_row d_col (d_col - 1) fp32 flops per layer; and the packed
+    output d_row d_col (1 + b/8) bytes per layer."""
     w = {"weights": 0, "syrk_flops": 0.0, "chol_flops": 0.0, "prop_flops": 0.0,
          "pack_bytes": 0.0}
     for layers in groups:
         d, n = layers[0].d_col, layers[0].n_tokens
         w["syrk_flops"] += float(d) * (d + 1) * n
-        w["chol_flops"] += 2.0 / 3.0 * float(d) ** 3
+        if route == "factor":
+            w["chol_flops"] += float(d) ** 3 / 3.0 + 128.0 * float(d) ** 2
+        else:
+            w["chol_flops"] += 2.0 / 3.0 * float(d) ** 3
         for s in layers:
             w["weights"] += s.d_row * s.d_col
             w["prop_flops"] += float(s.d_row) * s.d_col * (s.d_col - 1)
@@ -466,8 +478,14 @@ def run_ours(args, rank, world, local_rank):
     G.load_library()
     dev = torch.device("cuda", local_rank)
     groups = workload_layers(args.workload, rank, args.bits, args.sym, args.tokens)
-    work = work_model(groups)
+    work = work_model(groups, args.route)
     x_hosts, w_hosts = host_inputs(groups, pin=True)
+    factor = args.route == "factor"
+    if factor and any(s.block != 128 or (s.group and 128 % s.group) for g in groups for s in g):
+        raise SystemExit("--route factor needs block 128 and group_size 0 or a divisor of 128")
+    routes = {"factor": (G.gptq_prepare_factor, G.gptq_quantize_layer_factor),
+              "inverse": (G.gptq_prepare_hinv, G.gptq_quantize_layer)}
+    prepare, quantize = routes[args.route]
 
     cfgs = [[G.make_config(bits=s.bits, group_size=s.group, sym=s.sym, block=s.block,
                            damp_rel=s.damp) for s in layers] for layers in groups]
@@ -486,7 +504,9 @@ def run_ours(args, rank, world, local_rank):
                     for s, c in zip(layers, cfgs[gi])]})
     stream = torch.cuda.current_stream(dev)
 
-    def step(marks=None):
+    def step(marks=None, route=None):
+        prep, quant = routes[route or args.route]
+
         def mark(stage):
             if marks is not None:
                 e = torch.cuda.Event(enable_timing=True)
@@ -499,11 +519,11 @@ def run_ours(args, rank, world, local_rank):
             mark("zero_h")
             G.gptq_hessian_accumulate(b["H"], b["x"])
             mark("hessian")
-            G.gptq_prepare_hinv(b["H"], layers[0].damp, b["G"], b["dead"], ws)
+            prep(b["H"], layers[0].damp, b["G"], b["dead"], ws)
             mark("prepare")
             for li, s in enumerate(layers):
                 qw, sc, ze = b["out"][li]
-                G.gptq_quantize_layer(b["w"][li], b["G"], b["dead"], cfgs[gi][li], qw, sc, ze, ws)
+                quant(b["w"][li], b["G"], b["dead"], cfgs[gi][li], qw, sc, ze, ws)
                 mark("quantize")
 
     for _ in range(args.warmup):
@@ -540,11 +560,42 @@ def run_ours(args, rank, world, local_rank):
     ms_max = max_over_ranks(ms, world, dev)
     value = weak_value(world, work["weights"], ms_max)
 
+    # ---- the inverse route (G = chol(H^-1) whole) on the same inputs, for
+    # comparison: same warm-up, up to 5 timed steps, its own stage times
+    other = None
+    if factor and not args.no_other_route:
+        for _ in range(args.warmup):
+            step(route="inverse")
+        omarks = [[] for _ in range(min(args.steps, 5))]
+        o0, o1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        o0.record(stream)
+        for m in omarks:
+            step(m, route="inverse")
+        o1.record(stream)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        oms = max_over_ranks(o0.elapsed_time(o1) / len(omarks), world, dev)
+        ostage = {k: 0.0 for k in ("zero_h", "hessian", "prepare", "quantize")}
+        for m in omarks:
+            for (_, a), (stage, b) in zip(m[:-1], m[1:]):
+                ostage[stage] += a.elapsed_time(b) / len(omarks)
+        if G.gptq_device_status() != 0:
+            raise RuntimeError("device status set while timing the inverse route")
+        owork = work_model(groups, "inverse")
+        other = {"route": "inverse", "steps": len(omarks), "ms_per_step": oms,
+                 "value": weak_value(world, owork["weights"], oms), "unit": UNIT,
+                 "stage_ms": ostage,
+                 "prepare_tflops": owork["chol_flops"] / (ostage["prepare"] / 1e3) / 1e12}
+
     # ---- end to end: host buffers in, host buffers out, through the same API
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(args, G, groups, cfgs, x_hosts, w_hosts, dev_in, ws, dev, stream, world,
-                      work["weights"])
+                      work["weights"], prepare, quantize)
 
     if rank != 0:
         return
@@ -564,15 +615,18 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16 in / f32 acc (H); f64 (factor); f32 (sweep)",
         "data": "synthetic (seeded LLaMA-shaped layers and activations)",
-        "config": workload_config(args.workload, groups, world),
+        "config": dict(workload_config(args.workload, groups, world), route=args.route),
         "stage_ms": stage_ms, "stages": stages,
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": launches, "clocks": clk,
     }
+    if other is not None:
+        line["inverse_route"] = other
     print(json.dumps(line), flush=True)
 
 
-def run_e2e(args, G, groups, cfgs, x_hosts, w_hosts, dev_in, ws, dev, stream, world, weights):
+def run_e2e(args, G, groups, cfgs, x_hosts, w_hosts, dev_in, ws, dev, stream, world, weights,
+            prepare, quantize):
     """Same metric through the public API with host buffers: every step copies
     each X and each W from pinned host memory and reads the packed results
     back to the host.  The inputs are double-buffered on the device, and a
@@ -608,11 +662,10 @@ def run_e2e(args, G, groups, cfgs, x_hosts, w_hosts, dev_in, ws, dev, stream, wo
             b, inp = dev_in[gi], bufs[k][gi]
             b["H"].zero_()
             G.gptq_hessian_accumulate(b["H"], inp["x"])
-            G.gptq_prepare_hinv(b["H"], layers[0].damp, b["G"], b["dead"], ws)
+            prepare(b["H"], layers[0].damp, b["G"], b["dead"], ws)
             for li, s in enumerate(layers):
                 qw, sc, ze = b["out"][li]
-                G.gptq_quantize_layer(inp["w"][li], b["G"], b["dead"], cfgs[gi][li], qw, sc,
-                                      ze, ws)
+                quantize(inp["w"][li], b["G"], b["dead"], cfgs[gi][li], qw, sc, ze, ws)
                 for h, t in zip(host_out[gi][li], b["out"][li]):
                     h.copy_(t, non_blocking=True)
         consumed[k].record(stream)
@@ -810,7 +863,7 @@ def run_sharded(args, rank, world, local_rank):
     x = synth.gen_tokens(spec, t0, t1).to(dev)
     w = synth.gen_weight(spec)[r0:r1].contiguous().to(dev)
     stream = torch.cuda.current_stream(dev)
-    base = sharded.cuda_steps(cfg, spec.damp, world, dev)
+    base = sharded.cuda_steps(cfg, spec.damp, world, dev, route=args.route)
     marks = {}
 
     def timed(name, fn):

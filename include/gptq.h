@@ -172,6 +172,37 @@ gptq_status gptq_quantize_layer(const float* W, int64_t d_row, int64_t d_col,
                                 float* scales, uint8_t* zeros,
                                 void* ws, size_t ws_bytes, void* stream);
 
+/* The same quantized layer with half of the fp64 work of gptq_prepare_hinv:
+ * the column sweep never needs G = V^-1 outside its 128x128 diagonal
+ * blocks.  From the sweep's recurrence (dingiv.github.io page, section
+ * GPTQ: each column's error e_q = (w_q - w^_q)/G_qq is subtracted times row q
+ * of G), W = W^ + E G, so E = (W - W^) V.  The running weights at the start
+ * of 128-column block b are therefore
+ *   W_b + sum_{a<b} (W - W^)_a V_ab G_bb,
+ * the same values the sweep through G reaches there (the same sums in
+ * another order), and inside the block the sweep runs through G_bb as
+ * before.
+ * gptq_prepare_factor takes the arguments of gptq_prepare_hinv and writes
+ *  F  fp32 d x d: F_bb = G_bb on the diagonal 128-blocks (block b covers
+ *     columns [128 b, 128 b + 128), the last one ragged), F_ab = V_ab G_bb
+ *     for blocks a < b, 0 below the diagonal.
+ * It factors H' once (d^3/3 flops) and forms no inverse beyond the diagonal
+ * blocks; errors, pivots and synchronization as gptq_prepare_hinv.
+ * gptq_quantize_layer_factor takes the arguments of gptq_quantize_layer
+ * with F in place of G and writes the same outputs.  It needs
+ * cfg->block == 128 and group_size 0 or a divisor of 128 (a group's
+ * parameters are read from the running weights, which F gives exactly at
+ * block starts only); otherwise GPTQ_ERR_INVALID.  Asynchronous. */
+gptq_status gptq_prepare_factor(const float* H, int64_t d, double damp_rel,
+                                float* F, uint8_t* dead_mask,
+                                void* ws, size_t ws_bytes,
+                                int64_t* bad_pivot, void* stream);
+gptq_status gptq_quantize_layer_factor(const float* W, int64_t d_row, int64_t d_col,
+                                       const float* F, const uint8_t* dead_mask,
+                                       const gptq_config* cfg, uint32_t* qweight,
+                                       float* scales, uint8_t* zeros,
+                                       void* ws, size_t ws_bytes, void* stream);
+
 /* Dequantize the packed output and measure the layer loss of the page's
  * objective through the Hessian: loss = 1/2 * sum_r dW_r H dW_r^T with
  * dW = W - W^, which equals ||W X - W^ X||_F^2 for H = 2 X X^T

@@ -176,6 +176,51 @@ def _group_bounds(d_col: int, group: int):
     return [(c, min(c + g, d_col)) for c in range(0, d_col, g)]
 
 
+def factor_blocks(u: np.ndarray, block: int = 128) -> np.ndarray:
+    """``F`` for the sweep that never forms ``U`` outside its diagonal
+    blocks.  Reading of section GPTQ's recurrence: with ``e_q = (w_q -
+    w^_q) / U_qq`` and ``e_q U[q, k]`` subtracted from each later column,
+    the original weights are ``W = W^ + E U``, so ``E = (W - W^) V`` with
+    ``V = U^-1`` (upper, ``H' = V V^T``).  The running weights at the start
+    of block ``b`` are then ``W_b + sum_{a<b} (W - W^)_a V_ab U_bb``.
+    ``F`` holds ``U_bb`` on the diagonal blocks (``[block*b, block*b +
+    block)``, the last one ragged) and ``V_ab U_bb`` right of them, zero
+    below.  Parity unpinned by the pages (it is this reading); pinned by the
+    tests against ``gptq_quantize`` and the identity ``E = (W - W^) V``."""
+    u = np.asarray(u, dtype=F64)
+    d = u.shape[0]
+    v = np.linalg.inv(u)
+    f = np.zeros_like(u)
+    for b0 in range(0, d, block):
+        b1 = min(b0 + block, d)
+        f[b0:b1, b0:b1] = np.triu(u[b0:b1, b0:b1])
+        f[:b0, b0:b1] = v[:b0, b0:b1] @ u[b0:b1, b0:b1]
+    return f
+
+
+def factor_rows(u: np.ndarray, rows, block: int = 128) -> np.ndarray:
+    """Rows of ``factor_blocks(u, block)`` without inverting all of ``U``:
+    row ``i`` of ``V = U^-1`` solves ``U^T x = e_i`` (one triangular solve),
+    then ``F[i, b] = V[i, b] U_bb`` for the blocks right of ``i``'s and
+    ``U[i, b]`` in its own block."""
+    import scipy.linalg
+    u = np.asarray(u, dtype=F64)
+    d = u.shape[0]
+    rows = np.asarray(rows, dtype=np.int64)
+    rhs = np.zeros((d, rows.size), dtype=F64)
+    rhs[rows, np.arange(rows.size)] = 1.0
+    v_rows = scipy.linalg.solve_triangular(u, rhs, trans="T", lower=False).T
+    out = np.zeros((rows.size, d), dtype=F64)
+    for k, i in enumerate(rows):
+        b0 = (i // block) * block
+        b1 = min(b0 + block, d)
+        out[k, i:b1] = u[i, i:b1]
+        for c0 in range(b1, d, block):
+            c1 = min(c0 + block, d)
+            out[k, c0:c1] = v_rows[k, c0:c1] @ u[c0:c1, c0:c1]
+    return out
+
+
 # ---------------------------------------------------------------------------
 # GPTQ  (section GPTQ: fixed order, Cholesky of H^-1, blocks + lazy update)
 # ---------------------------------------------------------------------------

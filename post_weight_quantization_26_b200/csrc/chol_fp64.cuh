@@ -711,5 +711,41 @@ __global__ void write_g_kernel(const double* __restrict__ Mt, int d, float* __re
   }
 }
 
+// F (fp32, the sweep's order) from the blocks the factor route leaves in
+// Mt.  With V = J L J the upper factor of H' = V V^T and G = V^-1:
+//   inside a diagonal 128-block b:  F_bb = G_bb = (V_bb)^-1 = J X_kk J,
+//     read like G above (Mt's diagonal blocks hold X_kk^T);
+//   right of it (i < j, blocks a < b):  F_ab = V_ab G_bb, which is
+//     J (L_{>k,k} X_kk) J, left by the factorization in Mt's lower part:
+//     F[i][j] = Mt[d-1-i][d-1-j];
+//   below the diagonal: 0.
+// A 32 x 32 tile never straddles a 128-block boundary.
+__global__ void write_f_kernel(const double* __restrict__ Mt, int d, float* __restrict__ F) {
+  __shared__ double tile[32][33];
+  const int i0 = blockIdx.y * 32, j0 = blockIdx.x * 32;
+  const int tx = threadIdx.x, ty = threadIdx.y;  // 32 x 8
+  if (i0 / NB == j0 / NB) {  // diagonal block: as write_g_kernel
+    for (int yy = ty; yy < 32; yy += 8) {
+      const int j = j0 + yy, i = i0 + tx;
+      double v = 0.0;
+      if (j < d && i < d && i <= j) v = Mt[static_cast<long long>(d - 1 - j) * d + (d - 1 - i)];
+      tile[yy][tx] = v;
+    }
+    __syncthreads();
+    for (int yy = ty; yy < 32; yy += 8) {
+      const int i = i0 + yy, j = j0 + tx;
+      if (i < d && j < d) F[static_cast<long long>(i) * d + j] = static_cast<float>(tile[tx][yy]);
+    }
+    return;
+  }
+  for (int yy = ty; yy < 32; yy += 8) {
+    const int i = i0 + yy, j = j0 + tx;
+    if (i >= d || j >= d) continue;
+    const float v = (i0 < j0) ? static_cast<float>(Mt[static_cast<long long>(d - 1 - i) * d + (d - 1 - j)])
+                              : 0.0f;
+    F[static_cast<long long>(i) * d + j] = v;
+  }
+}
+
 }  // namespace chol
 }  // namespace gptq

@@ -133,6 +133,9 @@ gptq_status device_setup(int* num_sms) {
     GPTQ_CUDA_TRY(cudaFuncSetAttribute(quant::block_step_kernel<32>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        quant::block_step_smem<32>()));
+    GPTQ_CUDA_TRY(cudaFuncSetAttribute(quant::block_step_kernel<128, true>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       quant::block_step_smem<128>()));
     GPTQ_CUDA_TRY(cudaFuncSetAttribute(trail::trailing_tf32x3_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        trail::SMEM_BYTES));
@@ -144,6 +147,7 @@ gptq_status device_setup(int* num_sms) {
     for (const void* f : {reinterpret_cast<const void*>(quant::block_step_kernel<128>),
                           reinterpret_cast<const void*>(quant::block_step_kernel<64>),
                           reinterpret_cast<const void*>(quant::block_step_kernel<32>),
+                          reinterpret_cast<const void*>(quant::block_step_kernel<128, true>),
                           reinterpret_cast<const void*>(trail::trailing_tf32x3_kernel)})
       GPTQ_CUDA_TRY(cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout,
                                          cudaSharedmemCarveoutMaxShared));
@@ -641,9 +645,15 @@ gptq_status gptq_fault_inject(int where, int64_t wait_limit_ns) {
 }
 
 
-gptq_status gptq_prepare_hinv(const float* H, int64_t d, double damp_rel, float* G,
-                              uint8_t* dead_mask, void* ws, size_t ws_bytes,
-                              int64_t* bad_pivot, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The factorization behind gptq_prepare_hinv (factor = false: G = V^-1) and
+// gptq_prepare_factor (factor = true: F, see prepare_factor below).
+gptq_status prepare_impl(const float* H, int64_t d, double damp_rel, float* G,
+                         uint8_t* dead_mask, void* ws, size_t ws_bytes, int64_t* bad_pivot,
+                         void* stream, bool factor) {
   if (bad_pivot) *bad_pivot = -1;
   if (!H || !G || !dead_mask) return GPTQ_ERR_INVALID;
   if (d < 8 || d > 65536 || d % 8 != 0) return GPTQ_ERR_INVALID;
@@ -662,12 +672,22 @@ gptq_status gptq_prepare_hinv(const float* H, int64_t d, double damp_rel, float*
   double* Xd = reinterpret_cast<double*>(base + L.Xd);
   const int di = static_cast<int>(d);
   const int NB = chol::NB;
-  const int nt = (di + NB - 1) / NB;
+  // Block k covers [bstart(k), bstart(k+1)).  For F the blocks of the
+  // reversed matrix must map onto the sweep's blocks [128 b, 128 b + 128) of
+  // the original order, so a ragged block (d % 128 != 0) comes first rather
+  // than last.
+  const int shift = factor ? di % NB : 0;
+  const int nt = shift ? 1 + (di - shift) / NB : (di + NB - 1) / NB;
+  auto bstart = [&](int k) {
+    if (k >= nt) return di;
+    return shift ? (k == 0 ? 0 : shift + (k - 1) * NB) : k * NB;
+  };
   auto at = [&](double* m, int r, int c) { return m + static_cast<size_t>(r) * di + c; };
 
   GPTQ_CUDA_TRY(cudaMemsetAsync(pivot, 0xFF, 8, s));
-  // M^T accumulates its off-diagonal blocks from zero
-  GPTQ_CUDA_TRY(cudaMemsetAsync(Mt, 0, static_cast<size_t>(d) * d * 8, s));
+  // M^T accumulates its off-diagonal blocks from zero (F reads only the
+  // blocks it writes)
+  if (!factor) GPTQ_CUDA_TRY(cudaMemsetAsync(Mt, 0, static_cast<size_t>(d) * d * 8, s));
   chol::diag_stats_kernel<<<1, 1024, 0, s>>>(H, di, damp_rel, dead_mask, stats, istat);
   GPTQ_LAUNCH_CHECK();
   {
@@ -681,11 +701,12 @@ gptq_status gptq_prepare_hinv(const float* H, int64_t d, double damp_rel, float*
   cudaStream_t aux = dinfo->aux;
   cudaEvent_t evP[2] = {dinfo->ev[2], dinfo->ev[3]};
   cudaEvent_t evL[2] = {dinfo->ev[4], dinfo->ev[5]};
-  auto leaf = [&](int off, int n, cudaStream_t st) {
+  auto leaf = [&](int k, cudaStream_t st) {
+    const int off = bstart(k);
     chol::leaf_kernel<<<1, chol::LEAF_THREADS, chol::LEAF_SMEM, st>>>(
-        A, Mt, Xd + static_cast<size_t>(off / NB) * NB * NB, di, off, n, pivot);
+        A, Mt, Xd + static_cast<size_t>(k) * NB * NB, di, off, bstart(k + 1) - off, pivot);
   };
-  leaf(0, std::min(NB, di), s);
+  leaf(0, s);
   GPTQ_LAUNCH_CHECK();
   // Step k: P_k (caller's stream) forms the panel and rescales M's column
   // block k; then the auxiliary stream updates the next diagonal block (D_k)
@@ -695,9 +716,11 @@ gptq_status gptq_prepare_hinv(const float* H, int64_t d, double damp_rel, float*
   // remaining columns (K = one panel); the window's last panel updates every
   // column to its right with all m panels at once (K = 128 m), so most of the
   // d^3 work runs with long K.  m = 1 is the plain right-looking sweep.
+  // For F, M is not formed: its products are dropped, and U_k also writes
+  // the block row F_k = L_{>k,k} X_kk (see prepare_factor).
   const int m = chol::window_panels(di);
   for (int k = 0; k < nt; ++k) {
-    const int k0 = k * NB, nk = std::min(NB, di - k0), k1 = k0 + nk, rest = di - k1;
+    const int k0 = bstart(k), k1 = bstart(k + 1), nk = k1 - k0, rest = di - k1;
     double* Xk = Xd + static_cast<size_t>(k) * NB * NB;
     std::vector<chol::GemmProblem> pk;
     if (rest > 0) {
@@ -706,7 +729,7 @@ gptq_status gptq_prepare_hinv(const float* H, int64_t d, double damp_rel, float*
       q.M = rest; q.N = nk; q.K = nk; q.alpha = 1.0; q.beta = 0.0;
       pk.push_back(q);
     }
-    if (k0 > 0) {
+    if (k0 > 0 && !factor) {
       chol::GemmProblem q{};  // Mt[:k0, block k] <- Mt[:k0, block k] X_kk^T
       q.A = at(Mt, 0, k0); q.lda = di; q.B = Xk; q.ldb = NB; q.C = at(Mt, 0, k0); q.ldc = di;
       q.M = k0; q.N = nk; q.K = nk; q.alpha = 1.0; q.beta = 0.0;
@@ -715,15 +738,15 @@ gptq_status gptq_prepare_hinv(const float* H, int64_t d, double damp_rel, float*
     // 64-row tiles from about one wave of them up: the panel is K = 128
     // deep, so finer tiles balance the SMs better than 128-row ones (at
     // d = 22016, 342 tiles against 171 on 148 SMs)
-    const int prow = rest + k0;
+    const int prow = rest + (factor ? 0 : k0);
     if (prow >= 148 * 64) st = launch_nt<64, 2>(pk, s);
     else st = launch_nt<32, 1>(pk, s);
     if (st != GPTQ_OK) return st;
     if (rest <= 0) break;
-    const int n1 = std::min(NB, rest);  // next diagonal block
+    const int n1 = bstart(k + 2) - k1;  // next diagonal block
     // window of this panel: columns [e0, e1); the panels applied now are
     // [ka, k1) with K = kK, to the columns [k1, w1)
-    const int e0 = (k / m) * m * NB, e1 = std::min(di, e0 + m * NB);
+    const int e0 = bstart((k / m) * m), e1 = bstart((k / m) * m + m);
     const bool last = k1 >= e1;
     const int ka = last ? e0 : k0, kK = k1 - ka, w1 = last ? di : e1;
     GPTQ_CUDA_TRY(cudaEventRecord(evP[k & 1], s));
@@ -737,7 +760,7 @@ gptq_status gptq_prepare_hinv(const float* H, int64_t d, double damp_rel, float*
       q.M = n1; q.N = n1; q.K = kK; q.alpha = -1.0; q.beta = 1.0;
       st = launch_nt<32, 1>(dk, aux);
       if (st != GPTQ_OK) return st;
-      leaf(k1, n1, aux);
+      leaf(k + 1, aux);
       GPTQ_LAUNCH_CHECK();
       GPTQ_CUDA_TRY(cudaEventRecord(evL[k & 1], aux));
     }
@@ -764,11 +787,17 @@ gptq_status gptq_prepare_hinv(const float* H, int64_t d, double damp_rel, float*
         }
       }
     }
-    {
+    if (!factor) {
       chol::GemmProblem q{};  // Mt[:k1, k1:w1] -= Mt[:k1, ka:k1] L[k1:w1, ka:k1]^T
       q.A = at(Mt, 0, ka); q.lda = di; q.B = at(A, k1, ka); q.ldb = di;
       q.C = at(Mt, 0, k1); q.ldc = di;
       q.M = k1; q.N = w1 - k1; q.K = kK; q.alpha = -1.0; q.beta = 1.0;
+      uk.push_back(q);
+    } else {
+      chol::GemmProblem q{};  // F_k = L[k1:, k0:k1] X_kk into Mt's lower part
+      q.A = at(A, k1, k0); q.lda = di; q.B = at(Mt, k0, k0); q.ldb = di;  // X_kk^T
+      q.C = at(Mt, k1, k0); q.ldc = di;
+      q.M = rest; q.N = nk; q.K = nk; q.alpha = 1.0; q.beta = 0.0;
       uk.push_back(q);
     }
     // two SMs stay free for D_k and leaf k+1 on the auxiliary stream (the
@@ -779,7 +808,8 @@ gptq_status gptq_prepare_hinv(const float* H, int64_t d, double damp_rel, float*
   }
   {
     dim3 grid((di + 31) / 32, (di + 31) / 32);
-    chol::write_g_kernel<<<grid, dim3(32, 8), 0, s>>>(Mt, di, G);
+    if (factor) chol::write_f_kernel<<<grid, dim3(32, 8), 0, s>>>(Mt, di, G);
+    else chol::write_g_kernel<<<grid, dim3(32, 8), 0, s>>>(Mt, di, G);
     GPTQ_LAUNCH_CHECK();
   }
   long long host_pivot = -1;
@@ -793,15 +823,41 @@ gptq_status gptq_prepare_hinv(const float* H, int64_t d, double damp_rel, float*
   return GPTQ_OK;
 }
 
-gptq_status gptq_quantize_layer(const float* W, int64_t d_row, int64_t d_col, const float* G,
-                                const uint8_t* dead_mask, const gptq_config* cfg,
-                                uint32_t* qweight, float* scales, uint8_t* zeros, void* ws,
-                                size_t ws_bytes, void* stream) {
+}  // namespace
+
+extern "C" {
+
+gptq_status gptq_prepare_hinv(const float* H, int64_t d, double damp_rel, float* G,
+                              uint8_t* dead_mask, void* ws, size_t ws_bytes,
+                              int64_t* bad_pivot, void* stream) {
+  return prepare_impl(H, d, damp_rel, G, dead_mask, ws, ws_bytes, bad_pivot, stream, false);
+}
+
+gptq_status gptq_prepare_factor(const float* H, int64_t d, double damp_rel, float* F,
+                                uint8_t* dead_mask, void* ws, size_t ws_bytes,
+                                int64_t* bad_pivot, void* stream) {
+  return prepare_impl(H, d, damp_rel, F, dead_mask, ws, ws_bytes, bad_pivot, stream, true);
+}
+
+}  // extern "C"
+
+namespace {
+
+// The sweep behind gptq_quantize_layer (factor = false, G) and
+// gptq_quantize_layer_factor (factor = true, F).
+gptq_status quantize_impl(const float* W, int64_t d_row, int64_t d_col, const float* G,
+                          const uint8_t* dead_mask, const gptq_config* cfg, uint32_t* qweight,
+                          float* scales, uint8_t* zeros, void* ws, size_t ws_bytes, void* stream,
+                          bool factor) {
   if (!W || !G || !qweight || !scales || !zeros) return GPTQ_ERR_INVALID;
   if (d_row < 1 || d_row > (int64_t(1) << 24) || d_col < 32 || d_col % 32 != 0 ||
       d_col > 65536)
     return GPTQ_ERR_INVALID;
   if (!config_ok(cfg, d_col)) return GPTQ_ERR_INVALID;
+  // F's blocks are 128 wide, and a group's parameters must be taken inside
+  // one block (F gives the exact running weights only at block starts)
+  if (factor && (cfg->block != 128 || (cfg->group_size && 128 % cfg->group_size != 0)))
+    return GPTQ_ERR_INVALID;
   if (!aligned(W, 16) || !aligned(G, 16) || !aligned(qweight, 4) || !aligned(scales, 4))
     return GPTQ_ERR_INVALID;
   if (dead_mask && !aligned(dead_mask, 4)) return GPTQ_ERR_INVALID;
@@ -902,13 +958,15 @@ gptq_status gptq_quantize_layer(const float* W, int64_t d_row, int64_t d_col, co
     float* Ecf = Eb[cb][2] + pos * B;
     float* Ech = Eb[cb][0] + pos * B;
     float* Ecl = Eb[cb][1] + pos * B;
-#define GPTQ_STEP(BB)                                                                        \
-  quant::block_step_kernel<BB><<<qgrid, quant::QTHREADS, quant::block_step_smem<BB>(), s>>>( \
-      Wk, dr, dc, j0, ncols, G, Ep, jp0, nprev, lde, Ecf, Ech, Ecl, qweight, scales, zeros,     \
-      cfg->bits, cfg->sym, g, n_groups, per_channel)
-    if (B == 128) GPTQ_STEP(128);
-    else if (B == 64) GPTQ_STEP(64);
-    else GPTQ_STEP(32);
+#define GPTQ_STEP(BB, FAC)                                                                 \
+  quant::block_step_kernel<BB, FAC>                                                        \
+      <<<qgrid, quant::QTHREADS, quant::block_step_smem<BB>(), s>>>(                       \
+          Wk, dr, dc, j0, ncols, G, Ep, jp0, nprev, lde, Ecf, Ech, Ecl, qweight, scales,  \
+          zeros, cfg->bits, cfg->sym, g, n_groups, per_channel, W, dead_mask)
+    if (factor) GPTQ_STEP(128, true);
+    else if (B == 128) GPTQ_STEP(128, false);
+    else if (B == 64) GPTQ_STEP(64, false);
+    else GPTQ_STEP(32, false);
 #undef GPTQ_STEP
     GPTQ_LAUNCH_CHECK();
     GPTQ_CUDA_TRY(cudaEventRecord(evQ[jb % 4], s));
@@ -928,6 +986,26 @@ gptq_status gptq_quantize_layer(const float* W, int64_t d_row, int64_t d_col, co
   GPTQ_CUDA_TRY(cudaEventRecord(ev_join, di->aux));
   GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, ev_join, 0));
   return GPTQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+gptq_status gptq_quantize_layer(const float* W, int64_t d_row, int64_t d_col, const float* G,
+                                const uint8_t* dead_mask, const gptq_config* cfg,
+                                uint32_t* qweight, float* scales, uint8_t* zeros, void* ws,
+                                size_t ws_bytes, void* stream) {
+  return quantize_impl(W, d_row, d_col, G, dead_mask, cfg, qweight, scales, zeros, ws, ws_bytes,
+                       stream, false);
+}
+
+gptq_status gptq_quantize_layer_factor(const float* W, int64_t d_row, int64_t d_col,
+                                       const float* F, const uint8_t* dead_mask,
+                                       const gptq_config* cfg, uint32_t* qweight, float* scales,
+                                       uint8_t* zeros, void* ws, size_t ws_bytes, void* stream) {
+  return quantize_impl(W, d_row, d_col, F, dead_mask, cfg, qweight, scales, zeros, ws, ws_bytes,
+                       stream, true);
 }
 
 gptq_status gptq_dequant_check(const uint32_t* qweight, const float* scales, const uint8_t* zeros,

@@ -192,7 +192,11 @@ __device__ __forceinline__ void stage_gblock(float* dst, const float* G, int d_c
   }
 }
 
-template <int B>
+// FACTOR: G is the matrix F of gptq_prepare_factor (G's diagonal blocks,
+// V_ab G_bb right of them) and the errors written for the later blocks are
+// w^ - w_orig (Wo, the caller's weights, dead columns read as 0) instead of
+// e; inside the block the sweep is unchanged.
+template <int B, bool FACTOR = false>
 __global__ void __launch_bounds__(QTHREADS)
 block_step_kernel(const float* __restrict__ Wk, int d_row, int d_col, int j0, int ncols,
                   const float* __restrict__ G, const float* __restrict__ Eprev, int jp0,
@@ -200,7 +204,8 @@ block_step_kernel(const float* __restrict__ Wk, int d_row, int d_col, int j0, in
                   float* __restrict__ Ecur_lo,
                   uint32_t* __restrict__ qweight, float* __restrict__ scales,
                   uint8_t* __restrict__ zeros, int bits, int sym, int group, int n_groups,
-                  int pc_mode) {
+                  int pc_mode, const float* __restrict__ Wo,
+                  const uint8_t* __restrict__ dead) {
   using L = StepSmem<B>;
   constexpr int LDG = L::LDG;
   extern __shared__ __align__(16) uint8_t qsm[];
@@ -402,6 +407,7 @@ block_step_kernel(const float* __restrict__ Wk, int d_row, int d_col, int j0, in
         const float xh = s * (qf - z);
         const float e = (x - xh) * iv[u];
         ev[u] = e;
+        if (FACTOR) w[u] = xh;  // w[u] is not read again
         cw[u >> 2] |= static_cast<uint32_t>(qf) << (8 * (u & 3));
         // the later columns of the sub-block: w -= e G[q, later]
         const float* grow = Gs + (q0 + u) * LDG + q0;
@@ -419,6 +425,10 @@ block_step_kernel(const float* __restrict__ Wk, int d_row, int d_col, int j0, in
         *reinterpret_cast<float4*>(he + q0 + 4 * i) =
             make_float4(ev[4 * i], ev[4 * i + 1], ev[4 * i + 2], ev[4 * i + 3]);
         crow[q0 / 4 + i] = cw[i];
+        // the sub-block's own columns of W are no longer read: keep w^ there
+        if (FACTOR)
+          *reinterpret_cast<float4*>(hw + q0 + 4 * i) =
+              make_float4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
       }
       if (sb + 1 < nsb) named_bar_arrive(1, QTHREADS);
     }
@@ -475,9 +485,26 @@ block_step_kernel(const float* __restrict__ Wk, int d_row, int d_col, int j0, in
     float* ef = Ecur + static_cast<size_t>(r) * lde;
     float* eh = Ecur_hi + static_cast<size_t>(r) * lde;
     float* el = Ecur_lo + static_cast<size_t>(r) * lde;
+    const float* xrow = Ws + rloc * LDG;
+    const float* worow = FACTOR ? Wo + static_cast<size_t>(r) * d_col + j0 : nullptr;
     for (int c = 4 * t; c < B; c += 16) {
-      const float4 v = (c < ncols) ? *reinterpret_cast<const float4*>(erow + c)
-                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (c < ncols) {
+        if (FACTOR) {
+          const float4 xh = *reinterpret_cast<const float4*>(xrow + c);
+          float4 wo = *reinterpret_cast<const float4*>(worow + c);
+          if (dead) {
+            const uchar4 dm = *reinterpret_cast<const uchar4*>(dead + j0 + c);
+            if (dm.x) wo.x = 0.0f;
+            if (dm.y) wo.y = 0.0f;
+            if (dm.z) wo.z = 0.0f;
+            if (dm.w) wo.w = 0.0f;
+          }
+          v = make_float4(xh.x - wo.x, xh.y - wo.y, xh.z - wo.z, xh.w - wo.w);
+        } else {
+          v = *reinterpret_cast<const float4*>(erow + c);
+        }
+      }
       *reinterpret_cast<float4*>(ef + c) = v;
       const float4 h = make_float4(__uint_as_float(__float_as_uint(v.x) & 0xFFFFE000u),
                                    __uint_as_float(__float_as_uint(v.y) & 0xFFFFE000u),

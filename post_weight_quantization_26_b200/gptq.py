@@ -24,6 +24,7 @@ STATUS_NAMES = {0: "GPTQ_OK", 1: "GPTQ_ERR_INVALID", 2: "GPTQ_ERR_NOT_SPD",
 
 EXPORTED = ("gptq_workspace_size", "gptq_hessian_accumulate",
             "gptq_hessian_accumulate_ordered", "gptq_fault_inject", "gptq_prepare_hinv", "gptq_quantize_layer", "gptq_dequant_check",
+            "gptq_prepare_factor", "gptq_quantize_layer_factor",
             "gptq_device_status", "gptq_status_string", "gptq_launch_count",
             "gptq_dequant_check_noalloc", "gptq_w4a16_matmul", "gptq_awq_channel_scale",
             "gptq_awq_workspace_size", "gptq_awq_search")
@@ -78,6 +79,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gptq_quantize_layer.argtypes = [P, I64, I64, P, P, cfgp, P, P, P, P,
                                         SZ, P]
     lib.gptq_quantize_layer.restype = I
+    lib.gptq_prepare_factor.argtypes = lib.gptq_prepare_hinv.argtypes
+    lib.gptq_prepare_factor.restype = I
+    lib.gptq_quantize_layer_factor.argtypes = lib.gptq_quantize_layer.argtypes
+    lib.gptq_quantize_layer_factor.restype = I
     lib.gptq_dequant_check.argtypes = [P, P, P, P, P, I64, I64, cfgp, P,
                                        ctypes.POINTER(D), P, SZ, P]
     lib.gptq_dequant_check.restype = I
@@ -179,19 +184,51 @@ def gptq_prepare_hinv(H: torch.Tensor, damp_rel: float, G: torch.Tensor,
     return int(piv.value)
 
 
-def gptq_quantize_layer(W: torch.Tensor, G: torch.Tensor, dead_mask,
-                        cfg: GptqConfig, qweight: torch.Tensor,
-                        scales: torch.Tensor, zeros: torch.Tensor,
-                        ws: torch.Tensor, stream=None) -> None:
+def gptq_prepare_factor(H: torch.Tensor, damp_rel: float, F: torch.Tensor,
+                        dead_mask: torch.Tensor, ws: torch.Tensor,
+                        stream=None) -> int:
+    """F for gptq_quantize_layer_factor: G's 128x128 diagonal blocks and
+    V_ab G_bb right of them (H + damp = V V^T).  Returns bad_pivot."""
+    d = H.shape[0]
+    assert H.dtype == torch.float32 and H.shape == (d, d) and H.is_contiguous()
+    assert F.dtype == torch.float32 and F.shape == (d, d) and F.is_contiguous()
+    assert dead_mask.dtype == torch.uint8 and dead_mask.numel() == d
+    piv = ctypes.c_int64(-1)
+    st = load_library().gptq_prepare_factor(
+        _ptr(H), d, float(damp_rel), _ptr(F), _ptr(dead_mask), _ptr(ws),
+        ws.numel(), ctypes.byref(piv), _stream(stream))
+    _check(st, "gptq_prepare_factor", f" (bad_pivot={piv.value})")
+    return int(piv.value)
+
+
+def _quantize(name, W, G, dead_mask, cfg, qweight, scales, zeros, ws, stream):
     d_row, d_col = W.shape
     assert W.dtype == torch.float32 and W.is_contiguous()
     assert G.dtype == torch.float32 and G.shape == (d_col, d_col) and G.is_contiguous()
     assert qweight.dtype == torch.int32 or qweight.dtype == torch.uint32
-    st = load_library().gptq_quantize_layer(
+    st = getattr(load_library(), name)(
         _ptr(W), d_row, d_col, _ptr(G), _ptr(dead_mask), ctypes.byref(cfg),
         _ptr(qweight), _ptr(scales), _ptr(zeros), _ptr(ws), ws.numel(),
         _stream(stream))
-    _check(st, "gptq_quantize_layer")
+    _check(st, name)
+
+
+def gptq_quantize_layer(W: torch.Tensor, G: torch.Tensor, dead_mask,
+                        cfg: GptqConfig, qweight: torch.Tensor,
+                        scales: torch.Tensor, zeros: torch.Tensor,
+                        ws: torch.Tensor, stream=None) -> None:
+    _quantize("gptq_quantize_layer", W, G, dead_mask, cfg, qweight, scales,
+              zeros, ws, stream)
+
+
+def gptq_quantize_layer_factor(W: torch.Tensor, F: torch.Tensor, dead_mask,
+                               cfg: GptqConfig, qweight: torch.Tensor,
+                               scales: torch.Tensor, zeros: torch.Tensor,
+                               ws: torch.Tensor, stream=None) -> None:
+    """The same layer from F (gptq_prepare_factor); block 128, group_size 0
+    or a divisor of 128."""
+    _quantize("gptq_quantize_layer_factor", W, F, dead_mask, cfg, qweight,
+              scales, zeros, ws, stream)
 
 
 def gptq_dequant_check(qweight, scales, zeros, W, H, cfg: GptqConfig,

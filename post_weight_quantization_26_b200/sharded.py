@@ -5,10 +5,11 @@ GPTQ splits two ways (dingiv.github.io "量化" page, section GPTQ):
 * H = 2 X X^T is a sum over calibration tokens, so rank r accumulates H over
   its own token shard and one sum all-reduce gives every rank the full H.
   This is the path's only exchange step.
-* Given G, every row of W is quantized independently of the others, so
-  every rank factors the same H (the kernels are deterministic, so the
-  ranks get identical G and dead-channel masks, and nothing is broadcast)
-  and quantizes its own contiguous shard of rows.  The packed outputs are
+* Given G (or F, the factor route's matrix), every row of W is quantized
+  independently of the others, so every rank factors the same H (the
+  kernels are deterministic, so the ranks get identical matrices and
+  dead-channel masks, and nothing is broadcast) and quantizes its own
+  contiguous shard of rows.  The packed outputs are
   row-major, so gathering the shards in rank order gives the layer's
   output.
 
@@ -88,9 +89,10 @@ def gather_padded(t, world: int, device):
     return torch.cat([p[:r] for p, r in zip(parts, rows)], 0)
 
 
-def cuda_steps(cfg, damp: float, world: int, device=None) -> Steps:
+def cuda_steps(cfg, damp: float, world: int, device=None, route: str = "factor") -> Steps:
     """The library's kernels on this rank's GPU; NCCL collectives over the
-    default process group (none when ``world`` is 1)."""
+    default process group (none when ``world`` is 1).  ``route`` "factor"
+    prepares F and sweeps through it; "inverse" prepares G = chol(H^-1)."""
     import torch
     import torch.distributed as dist
 
@@ -98,6 +100,10 @@ def cuda_steps(cfg, damp: float, world: int, device=None) -> Steps:
 
     G.load_library()  # fails loudly without the library: there is no other path
     dev = torch.device(device or "cuda")
+    if route not in ("factor", "inverse"):
+        raise ValueError(f"unknown route {route!r}")
+    prep = G.gptq_prepare_factor if route == "factor" else G.gptq_prepare_hinv
+    quant = G.gptq_quantize_layer_factor if route == "factor" else G.gptq_quantize_layer
 
     def zeros_h(d):
         return torch.zeros((d, d), dtype=torch.float32, device=dev)
@@ -114,7 +120,7 @@ def cuda_steps(cfg, damp: float, world: int, device=None) -> Steps:
         g = torch.empty_like(H)
         dead = torch.empty(d, dtype=torch.uint8, device=dev)
         ws = G.alloc_workspace(1, d, cfg, device=dev)
-        G.gptq_prepare_hinv(H, damp, g, dead, ws)
+        prep(H, damp, g, dead, ws)
         return g, dead
 
     def quantize(w, g, dead):
@@ -122,7 +128,7 @@ def cuda_steps(cfg, damp: float, world: int, device=None) -> Steps:
         qw, sc, ze = G.alloc_outputs(d_row, d_col, cfg, device=dev)
         if d_row:
             ws = G.alloc_workspace(d_row, d_col, cfg, device=dev)
-            G.gptq_quantize_layer(w, g, dead, cfg, qw, sc, ze, ws)
+            quant(w, g, dead, cfg, qw, sc, ze, ws)
         return qw, sc, ze
 
     def allgather_rows(t):

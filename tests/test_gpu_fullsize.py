@@ -17,6 +17,10 @@ plain fp64 one (integer decisions in fp64); the bars are those of
   default benchmark layer) at 4 and 3 bits: the same, with the oracle's H
   (1.3e14 fp64 flops on the host) and its factor of that size.
 Every returned G is also checked by U^T U H' v = v on random vectors v.
+The q_proj, down_proj and 65B down projection layers are also quantized
+through the factor route (gptq_prepare_factor, gptq_quantize_layer_factor)
+and held to the same oracle layer, and rows of that route's F to the
+oracle's.
 """
 import numpy as np
 import pytest
@@ -84,11 +88,20 @@ def _gpu_prepare(G, h, spec, d_row_max):
     return g, dead, ws
 
 
-def _gpu_quantize(G, spec, w_host, g, dead, ws, h):
+def _gpu_prepare_factor(G, h, spec, ws):
+    f = torch.empty_like(h)
+    dead = torch.empty(spec.d_col, dtype=torch.uint8, device="cuda")
+    assert G.gptq_prepare_factor(h, spec.damp, f, dead, ws) == -1
+    assert not bool(dead.any())
+    return f, dead
+
+
+def _gpu_quantize(G, spec, w_host, g, dead, ws, h, factor=False):
     cfg = _cfg(G, spec)
     w = w_host.cuda()
     qw, sc, ze = G.alloc_outputs(spec.d_row, spec.d_col, cfg)
-    G.gptq_quantize_layer(w, g, dead, cfg, qw, sc, ze, ws)
+    quantize = G.gptq_quantize_layer_factor if factor else G.gptq_quantize_layer
+    quantize(w, g, dead, cfg, qw, sc, ze, ws)
     w_hat = torch.empty_like(w)
     loss = G.gptq_dequant_check(qw, sc, ze, w, h, cfg, W_hat=w_hat, ws=ws)
     assert G.gptq_device_status() == 0
@@ -167,39 +180,59 @@ def _sample_rows(d_row, seed, n=48):
 def _check_sampled_rows(spec, w_host, out, u, dead, h_ref, seed):
     """The oracle quantizes the sampled rows with its own factor; they are
     compared with the GPU's rows code by code, and their loss (through the
-    oracle's H) within the loss bar."""
+    oracle's H) within the loss bar.  `out` may be a list of GPU layers (the
+    two routes), all checked against the one oracle sweep."""
     rows = _sample_rows(spec.d_row, seed)
     w0 = w_host[torch.as_tensor(rows)].double().numpy()
     codes, scales, zeros, w_hat, _ = O.gptq_quantize(
         w0, u, spec.bits, spec.group, spec.sym, spec.block, dead=dead)
-    res = check_layer(_codes(out, spec, rows), _rows(out, "sc", rows), _rows(out, "ze", rows),
-                      codes, scales, zeros, spec.group)
     loss_ref = O.layer_loss_hessian(w0, w_hat, h_ref)
-    loss_gpu = O.layer_loss_hessian(w0, _rows(out, "w_hat", rows), h_ref)
-    check_loss(loss_gpu, loss_ref)
+    res = []
+    for o in (out if isinstance(out, list) else [out]):
+        res.append(check_layer(_codes(o, spec, rows), _rows(o, "sc", rows), _rows(o, "ze", rows),
+                               codes, scales, zeros, spec.group))
+        check_loss(O.layer_loss_hessian(w0, _rows(o, "w_hat", rows), h_ref), loss_ref)
     return res
+
+
+def _check_f_rows(f_dev, u, seed, n=24):
+    """Sampled rows of the GPU's F (gptq_prepare_factor) against the
+    oracle's rows of F from its own U."""
+    d = u.shape[0]
+    rng = np.random.default_rng(seed)
+    rows = np.unique(np.concatenate([[0, 127, 128, d - 1], rng.choice(d, n, replace=False)]))
+    got = f_dev[torch.as_tensor(rows, device=f_dev.device)].double().cpu().numpy()
+    ref = O.factor_rows(u, rows)
+    np.testing.assert_allclose(got, ref, rtol=1e-5, atol=1e-6 * np.abs(ref).max())
 
 
 # ------------------------------------- q_proj and down_proj: the whole oracle
 @pytest.mark.parametrize("spec", [synth.Q_PROJ_7B, synth.DOWN_PROJ_7B], ids=lambda s: s.name)
 def test_full_size_against_whole_oracle(G, spec):
+    """Both routes (G, and F from gptq_prepare_factor) against the whole
+    oracle; F itself against the oracle's F of its own U."""
     x, w = _inputs(spec)
     h = _gpu_hessian(G, x)
     g, dead, ws = _gpu_prepare(G, h, spec, spec.d_row)
     out = _gpu_quantize(G, spec, w, g, dead, ws, h)
     _check_g_property(h, g, spec.damp, seed=1)
+    del g
+    f, dead_f = _gpu_prepare_factor(G, h, spec, ws)
+    out_f = _gpu_quantize(G, spec, w, f, dead_f, ws, h, factor=True)
     h_ref = O.hessian(_Tokens(x))
     del x
     _check_h_whole(h, h_ref)
-    del h, g, dead, ws
+    del h, dead, dead_f, ws
     _free()
     ref = O.gptq(w.double().numpy(), h_ref, bits=spec.bits, group=spec.group,
                  sym=spec.sym, block=spec.block, damp_rel=spec.damp)
-    check_layer(_codes(out, spec), out["sc"].cpu().numpy(), out["ze"].cpu().numpy(),
-                ref["codes"], ref["scales"], ref["zeros"], spec.group)
     loss_ref = O.layer_loss_hessian(w.double().numpy(), ref["w_hat"], h_ref)
-    check_loss(out["loss"], loss_ref)
-    del out
+    for o in (out, out_f):
+        check_layer(_codes(o, spec), o["sc"].cpu().numpy(), o["ze"].cpu().numpy(),
+                    ref["codes"], ref["scales"], ref["zeros"], spec.group)
+        check_loss(o["loss"], loss_ref)
+    _check_f_rows(f, ref["u"], seed=2)
+    del out, out_f, f
     _free()
 
 
@@ -264,24 +297,32 @@ def test_mlp_65b_gate_up_against_oracle(G):
 
 def test_mlp_65b_down_proj_4_and_3_bits(G):
     """The 65B down projection (H of 22016^2, the default benchmark layer):
-    one accumulate and prepare on the GPU, then the layer at 4 and at 3 bits.
-    The oracle forms its own H from the tokens (checked whole against the
-    GPU's), its own factor, and quantizes sampled rows of both widths."""
+    one accumulate on the GPU, both prepares (G and F), then the layer at 4
+    and at 3 bits through each.  The oracle forms its own H from the tokens
+    (checked whole against the GPU's), its own factor, rows of F from it,
+    and quantizes sampled rows of both widths, checked against both
+    routes."""
     spec4 = [s for s, i in synth.mlp_65b(4) if i == 1][0]
     spec3 = [s for s, i in synth.mlp_65b(3) if i == 1][0]
     x, w = _inputs(spec4)
     h = _gpu_hessian(G, x)
     g, dead, ws = _gpu_prepare(G, h, spec4, spec4.d_row)
     _check_g_property(h, g, spec4.damp, seed=44)
-    outs = {spec.bits: _gpu_quantize(G, spec, w, g, dead, ws, h) for spec in (spec4, spec3)}
+    outs = {spec.bits: [_gpu_quantize(G, spec, w, g, dead, ws, h)] for spec in (spec4, spec3)}
+    del g
+    f, dead_f = _gpu_prepare_factor(G, h, spec4, ws)
+    for spec in (spec4, spec3):
+        outs[spec.bits].append(_gpu_quantize(G, spec, w, f, dead_f, ws, h, factor=True))
     h_ref = O.hessian(_Tokens(x))
     del x
     _check_h_whole(h, h_ref)
-    del h, g, dead, ws
+    del h, dead, dead_f, ws
     _free()
     hd, dead_ref = O.dampen(h_ref, spec4.damp)
     u = O.hinv_cholesky_upper(hd)
     del hd
+    _check_f_rows(f, u, seed=45)
+    del f
     for spec in (spec4, spec3):
         _check_sampled_rows(spec, w, outs[spec.bits], u, dead_ref, h_ref, seed=440 + spec.bits)
     del outs, u, h_ref

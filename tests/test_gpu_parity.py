@@ -223,6 +223,40 @@ def test_quantize_wide_layers_lazy_windows(G, case):
     check_layer(codes, sc, ze, ref_codes, ref_s, ref_z, group)
 
 
+@pytest.mark.parametrize("group", [0, 32, 128])
+def test_quantize_degenerate_rows(G, group):
+    """Rows the quantizer treats specially or that stress fp32 range: all zero
+    (min = max, the +-1 range of the quantizer's rule), constant of either
+    sign, one spike after zeros, a zero first half, and whole rows scaled by
+    1e-4 and by 1e4, quantized with a real factor, against the plain fp64
+    oracle.  (A group that holds nothing but the rounding residue of an
+    earlier column has parameters fitted to that residue, which fp32 and
+    fp64 leave at unrelated magnitudes; no row here makes one.)"""
+    d_row, d_col = 40, 256
+    spec = synth.tiny_spec(d_row, d_col, 4 * d_col, seed=900 + group)
+    w = synth.gen_weight(spec).numpy().astype(np.float64)
+    w[0] = 0.0
+    w[1] = 0.03
+    w[2] = -0.02
+    w[3] = 0.0
+    w[3, d_col - 5] = 0.5             # a spike in the last group: no group to its
+                                      # right holds only its rounding residue
+    w[4] *= 1e-4
+    w[5] *= 1e4
+    w[6, : d_col // 2] = 0.0          # a zero first half, then ordinary values
+    w = w.astype(np.float32)
+    h = O.hessian(synth.gen_tokens(spec).float().numpy())
+    hd, _ = O.dampen(h, 0.01)
+    u32 = np.ascontiguousarray(O.hinv_cholesky_upper(hd), dtype=np.float32)
+    codes, sc, ze, _ = _run_quantize(G, w, u32, 4, group, False, 128)
+    ref_codes, ref_s, ref_z, _, _ = O.gptq_quantize(
+        w.astype(np.float64), u32.astype(np.float64), 4, group, False, 128)
+    check_layer(codes, sc, ze, ref_codes, ref_s, ref_z, group)
+    assert np.all(np.isfinite(sc)) and np.all(sc > 0)
+    # an all-zero row stays at its zero point: nothing to propagate
+    assert np.all(codes[0] == ze[0, 0])
+
+
 def test_quantize_scaled_identity_is_rtn(G):
     """With G = c I nothing propagates: GPU output equals round-to-nearest."""
     spec = synth.tiny_spec(64, 256, 16)

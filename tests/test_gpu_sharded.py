@@ -24,12 +24,16 @@ def G():
     return gptq
 
 
-def test_one_rank_sequence_equals_the_direct_calls(G):
+@pytest.mark.parametrize("route", ["factor", "inverse"])
+def test_one_rank_sequence_equals_the_direct_calls(G, route):
     from post_weight_quantization_26_b200 import sharded
     spec = synth.tiny_spec(96, 512, 3000, seed=8).with_(group=128)
     cfg = G.make_config(bits=4, group_size=128)
     x, w = synth.gen_tokens(spec).cuda(), synth.gen_weight(spec).cuda()
-    qw, sc, ze, H = sharded.quantize_layer_sharded(sharded.cuda_steps(cfg, 0.01, 1), x, w, 512)
+    qw, sc, ze, H = sharded.quantize_layer_sharded(
+        sharded.cuda_steps(cfg, 0.01, 1, route=route), x, w, 512)
+    prep = G.gptq_prepare_factor if route == "factor" else G.gptq_prepare_hinv
+    quant = G.gptq_quantize_layer_factor if route == "factor" else G.gptq_quantize_layer
     # the direct calls
     h = torch.zeros((512, 512), dtype=torch.float32, device="cuda")
     g = torch.empty_like(h)
@@ -37,8 +41,8 @@ def test_one_rank_sequence_equals_the_direct_calls(G):
     ws = G.alloc_workspace(96, 512, cfg)
     q2, s2, z2 = G.alloc_outputs(96, 512, cfg)
     G.gptq_hessian_accumulate(h, x)
-    G.gptq_prepare_hinv(h, 0.01, g, dead, ws)
-    G.gptq_quantize_layer(w, g, dead, cfg, q2, s2, z2, ws)
+    prep(h, 0.01, g, dead, ws)
+    quant(w, g, dead, cfg, q2, s2, z2, ws)
     torch.cuda.synchronize()
     assert G.gptq_device_status() == 0
     # the Hessian's tiles are summed by TMA reduce-add in a run-dependent
