@@ -395,7 +395,8 @@ def kernel_traffic(name: str, src_rel: str):
         return None
 
 
-def stage_roofline(work, stage_ms, ms, peaks, peak_src, clk, groups, name, timed_ms):
+def stage_roofline(work, stage_ms, ms, peaks, peak_src, clk, groups, name, timed_ms,
+                   route="factor"):
     """Each stage against its own bound, the combined roofline T*, and the
     roofline object of the stage that takes the most time.  The bf16 peak is
     the measured burst figure when the timed region is shorter than a second
@@ -450,7 +451,8 @@ def stage_roofline(work, stage_ms, ms, peaks, peak_src, clk, groups, name, timed
                                              "prepare stage (with leaf_kernel and the damping)",
                 "achieved": ach["prepare"], "peak": fp64, "unit": "TFLOP/s",
                 "frac": ach["prepare"] / fp64,
-                "traffic": kernel_traffic(f"dgemm_nt_kernel/{name}",
+                "traffic": kernel_traffic(f"dgemm_nt_kernel/{name}" +
+                                          ("/factor" if route == "factor" else ""),
                                           "post_weight_quantization_26_b200/csrc/chol_fp64.cuh"),
                 "peak_source": f"derived: {SM_COUNT} SMs x 64 fp64 FMA/clk x 2 at the sampled "
                                f"{sm_mhz:.0f} MHz (no measured fp64 peak)"}
@@ -601,7 +603,7 @@ def run_ours(args, rank, world, local_rank):
         return
     peaks, peak_src = load_peaks()
     stages, roofline = stage_roofline(work, stage_ms, ms, peaks, peak_src, clk, groups,
-                                      args.workload, ms * args.steps)
+                                      args.workload, ms * args.steps, args.route)
     cpu = None
     if not args.no_cpu_baseline and world == 1:
         res = oracle_sample(groups, x_hosts, w_hosts, tokens=4096, fac_dim=8192, rows=32)

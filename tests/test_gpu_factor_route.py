@@ -153,11 +153,12 @@ def _wide(d_col):
 
 
 @pytest.mark.parametrize("case", [(48, 8448, 4, 128, False), (40, 8448, 3, 0, False),
-                                  (24, 8448, 4, 32, True)],
+                                  (24, 8448, 4, 32, True), (32, 8224, 4, 128, False)],
                          ids=lambda c: "x".join(map(str, c)))
 def test_quantize_factor_wide_layers_lazy_windows(G, case):
     """Windows of 4 blocks: inside one, each block's errors reach the
     window's later blocks; the window's errors reach the rest at once.
+    8224 columns end in a ragged block of 32 inside a part-full window.
     Layers of 24 to 48 rows: one row is 2-4% of the items, so a single tie
     at fp32 resolution (about one per million decisions on either route)
     would spend the pooled budget by itself.  Each row is therefore held to

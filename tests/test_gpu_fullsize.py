@@ -149,6 +149,38 @@ def _check_g_property(h_dev, g_dev, damp, seed):
     return hu, gu
 
 
+def _check_f_property(h_dev, f_dev, damp, seed, block=128):
+    """F from gptq_prepare_factor holds G_bb on its diagonal blocks and
+    V_ab G_bb right of them (H' = V V^T, G = V^-1).  G is applied through F
+    without forming it, as the sweep does, and G H' G^T v = v is checked on
+    random vectors v (the check of G above, in the form G H' G^T = I):
+      x = G^T v:  x_b = F_bb^T v_b - F[:b0, b]^T x[:b0]  (block columns, forward)
+      z = G y:    w_b = y_b - F[b, >b] w[>b],  z_b = F_bb w_b  (block rows, backward)"""
+    d = h_dev.shape[0]
+    assert float(torch.tril(f_dev, -1).abs().max()) == 0.0
+    assert bool((torch.diagonal(f_dev) > 0).all())
+    hu = h_dev.cpu().numpy()
+    fu = f_dev.cpu().numpy()
+    lam = damp * float(np.mean(np.diag(hu).astype(np.float64)))
+    v = np.random.default_rng(seed).standard_normal((d, 2))
+    starts = list(range(0, d, block))
+    x = np.zeros_like(v)
+    for b0 in starts:
+        b1 = min(b0 + block, d)
+        x[b0:b1] = (fu[b0:b1, b0:b1].astype(np.float64).T @ v[b0:b1]
+                    - fu[:b0, b0:b1].astype(np.float64).T @ x[:b0])
+    y = _sym_upper_matmul(hu, x) + lam * x
+    del hu
+    w = np.zeros_like(v)
+    z = np.zeros_like(v)
+    for b0 in reversed(starts):
+        b1 = min(b0 + block, d)
+        w[b0:b1] = y[b0:b1] - fu[b0:b1, b1:].astype(np.float64) @ w[b1:]
+        z[b0:b1] = fu[b0:b1, b0:b1].astype(np.float64) @ w[b0:b1]
+    rel = np.linalg.norm(z - v, axis=0) / np.linalg.norm(v, axis=0)
+    assert rel.max() <= G_RESID, f"G H' G^T v - v through F: rel {rel.max():.2e}"
+
+
 def _free():
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
@@ -311,6 +343,7 @@ def test_mlp_65b_down_proj_4_and_3_bits(G):
     outs = {spec.bits: [_gpu_quantize(G, spec, w, g, dead, ws, h)] for spec in (spec4, spec3)}
     del g
     f, dead_f = _gpu_prepare_factor(G, h, spec4, ws)
+    _check_f_property(h, f, spec4.damp, seed=46)
     for spec in (spec4, spec3):
         outs[spec.bits].append(_gpu_quantize(G, spec, w, f, dead_f, ws, h, factor=True))
     h_ref = O.hessian(_Tokens(x))

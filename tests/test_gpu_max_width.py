@@ -4,7 +4,8 @@ working copies needs 64 bits.
 
 * Hessian: sampled rows against the oracle's rows of H from the tokens.
 * Factor: U^T U H' v = v on random vectors (the oracle cannot factor a
-  65536^2 matrix in a test's time).
+  65536^2 matrix in a test's time), and for the factor route's F the same
+  identity with G applied through F.
 * Sweep: with G = c I nothing propagates, so the layer is round-to-nearest:
   within the stated bars of the fp64 oracle's, and exactly the oracle's
   when that takes its decisions in fp32 as the kernel does.
@@ -62,22 +63,35 @@ def test_max_width_hessian_and_factor(G):
     del ws
     torch.cuda.empty_cache()
     T._check_g_property(h, g, 0.01, seed=65)
-    del h, g, dead
+    del g
+    torch.cuda.empty_cache()
+    # the factor route's F at the same width
+    ws = G.alloc_workspace(8, D, cfg)
+    f = torch.empty_like(h)
+    assert G.gptq_prepare_factor(h, 0.01, f, dead, ws) == -1
+    assert G.gptq_device_status() == 0
+    del ws
+    torch.cuda.empty_cache()
+    T._check_f_property(h, f, 0.01, seed=66)
+    del h, f, dead
     torch.cuda.empty_cache()
 
 
-def test_max_width_sweep_identity_is_rtn(G):
+@pytest.mark.parametrize("route", ["inverse", "factor"])
+def test_max_width_sweep_identity_is_rtn(G, route):
+    """G = cI (and F = cI, the factor route's matrix for H' = c^-2 I)."""
     torch.cuda.empty_cache()
     d_row = 40
     spec = synth.tiny_spec(d_row, D, 8, seed=66)
     w = synth.gen_weight(spec).numpy()
     c = 1.0 / np.sqrt(5.05)
     g = torch.eye(D, dtype=torch.float32, device="cuda") * c
+    quantize = G.gptq_quantize_layer_factor if route == "factor" else G.gptq_quantize_layer
     for bits, group in ((4, 128), (3, 0)):
         cfg = G.make_config(bits=bits, group_size=group)
         qw, sc, ze = G.alloc_outputs(d_row, D, cfg)
         ws = G.alloc_workspace(d_row, D, cfg)
-        G.gptq_quantize_layer(torch.from_numpy(w).cuda(), g, None, cfg, qw, sc, ze, ws)
+        quantize(torch.from_numpy(w).cuda(), g, None, cfg, qw, sc, ze, ws)
         torch.cuda.synchronize()
         assert G.gptq_device_status() == 0
         codes = O.unpack_codes(qw.cpu().numpy().view(np.uint32), bits, D)
