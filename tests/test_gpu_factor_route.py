@@ -153,7 +153,7 @@ def _wide(d_col):
 
 
 @pytest.mark.parametrize("case", [(48, 8448, 4, 128, False), (40, 8448, 3, 0, False),
-                                  (24, 8448, 4, 32, True), (32, 8224, 4, 128, False)],
+                                  (24, 8448, 4, 32, True), (32, 8224, 4, 0, False)],
                          ids=lambda c: "x".join(map(str, c)))
 def test_quantize_factor_wide_layers_lazy_windows(G, case):
     """Windows of 4 blocks: inside one, each block's errors reach the
