@@ -40,7 +40,13 @@ diagonal; a dead input channel (``H_ii = 0``) gets ``H'_ii = 1`` and its
 weight column is zeroed.
 
 Every function here is pinned by ``tests/test_oracle.py`` against closed
-forms, invariants, brute force and hand-worked cases.
+forms, invariants, brute force and hand-worked cases, except
+``factor_blocks`` and ``factor_rows``: they define F for the sweep that
+needs U only on its diagonal blocks, a reading of section GPTQ's
+recurrence rather than a step the page prints, so the pages leave their
+parity unpinned; ``tests/test_oracle_factor.py`` pins them against this
+module's own sweep through U (and planted mistakes), the reversed-route
+Cholesky and closed forms.
 """
 from __future__ import annotations
 
