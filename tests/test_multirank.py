@@ -102,3 +102,21 @@ def test_workloads_group_layers_by_input():
     down = bench.workload_layers("down_proj_65b")
     assert [(s.d_row, s.d_col, s.n_tokens, s.group) for g in down for s in g] == \
         [(8192, 22016, 131072, 128)]
+
+
+def test_work_model_counts_each_route_work():
+    """The prepare stage's fp64 work per input: 2/3 d^3 on the inverse route
+    (Cholesky d^3/3 and triangular inverse d^3/3), d^3/3 + 128 d^2 on the
+    factor route (the Cholesky and the panels V_ab G_bb); the other stages
+    are the same on both."""
+    sys.path.insert(0, ROOT)
+    import bench
+    mlp = bench.workload_layers("mlp_65b")           # inputs of d = 8192 and 22016
+    inv = bench.work_model(mlp, "inverse")
+    fac = bench.work_model(mlp, "factor")
+    ds = [8192.0, 22016.0]
+    assert inv["chol_flops"] == pytest.approx(sum(2 * d ** 3 / 3 for d in ds))
+    assert fac["chol_flops"] == pytest.approx(sum(d ** 3 / 3 + 128 * d ** 2 for d in ds))
+    for k in ("weights", "syrk_flops", "prop_flops", "pack_bytes"):
+        assert inv[k] == fac[k]
+    assert bench.work_model(mlp) == inv                 # the model's default argument
