@@ -134,6 +134,29 @@ def test_prepare_and_quantize_validation(lib):
                                   1 << 20, None) == 1
 
 
+def test_factor_route_validation(lib):
+    """The factor route's calls take the same arguments and checks as the
+    inverse route's, and the sweep also rejects what F cannot serve: a block
+    other than 128 and a group size that does not divide 128."""
+    from post_weight_quantization_26_b200 import gptq as G
+    piv = ctypes.c_int64(123)
+    p = lib.gptq_prepare_factor
+    assert p(FAKE, 60, 0.01, FAKE, FAKE, FAKE, 1 << 30, ctypes.byref(piv), None) == 1
+    assert piv.value == -1
+    assert p(FAKE, 64, 0.01, FAKE, FAKE, None, 1 << 30, None, None) == 4
+    assert p(FAKE, 64, float("nan"), FAKE, FAKE, FAKE, 1 << 30, None, None) == 1
+    q = lib.gptq_quantize_layer_factor
+    for block, group in ((64, 0), (32, 32), (128, 256)):
+        cfg = G.make_config(group_size=group, block=block)
+        assert q(FAKE, 64, 512, FAKE, None, ctypes.byref(cfg), FAKE, FAKE, FAKE,
+                 FAKE, 1 << 30, None) == 1, (block, group)
+    cfg = G.make_config(group_size=32)
+    assert q(FAKE, 64, 100, FAKE, None, ctypes.byref(cfg), FAKE, FAKE, FAKE,
+             FAKE, 1 << 30, None) == 1
+    assert q(FAKE, 64, 512, FAKE, None, ctypes.byref(cfg), FAKE, FAKE, FAKE,
+             FAKE, 8, None) == 4
+
+
 def test_w4a16_matmul_validation(lib):
     """Rejected before any launch: other widths, batches, shapes, alignment."""
     from post_weight_quantization_26_b200 import gptq as G
