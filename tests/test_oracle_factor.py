@@ -163,3 +163,17 @@ def test_factor_rows_match_blocks(d):
     rows = np.array([0, 1, 127, 128, d // 2, d - 33, d - 1])
     got = O.factor_rows(u, rows)
     np.testing.assert_allclose(got, f[rows], rtol=1e-9, atol=1e-12 * np.abs(f).max())
+
+
+def test_groups_wider_than_a_block_need_the_running_weights_of_g():
+    """Why the factor route takes only group sizes that divide 128: a group
+    of 256 reads its parameters at its first column from the running weights
+    of both its blocks, and right of the current block F gives other partial
+    sums than U (only the full sums at a block start agree).  The scales of
+    the second group of 256 then differ from the oracle's."""
+    w, hd, _ = _layer(8, 24, 512, 2048)
+    u = O.hinv_cholesky_upper(hd)
+    ref = O.gptq_quantize(w, u, 4, 256, False, 128)
+    got = _sweep_factor(w, O.factor_blocks(u), 4, 256, False)
+    np.testing.assert_allclose(got[1][:, 0], ref[1][:, 0], rtol=1e-12)  # read from W itself
+    assert np.abs(got[1][:, 1] - ref[1][:, 1]).max() > 1e-6 * np.abs(ref[1][:, 1]).max()
